@@ -1,0 +1,542 @@
+"""Benchmark of the LightTransfer-Test prefill hot path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config gqa1p2b] [--impl ours|reference]
+
+One step is one pass of the whole path over one prefill of the workload: for
+every layer the causal GQA attention with LSE (lt_prefill_attn), the lazy ratio
+from that LSE (lt_lazy_ratio), the layer priority queue (lt_queue_push, host)
+and, for each layer the queue demotes, the KV compaction (lt_compact_kv).  The
+per-layer Q/K/V of all layers are resident in HBM before timing (together far
+larger than the 126 MB L2, so no L2 flush is needed between steps).  The ratio
+of layer l is read back asynchronously and pushed while layer l+1's attention
+runs, so the queue never stalls the GPU.
+
+Rank 0 prints one JSON line.  With --gpus N > 1 (torchrun) every rank runs an
+independent replica of the workload (the path has no exchange step): weak
+scaling, value = work of all ranks / max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "prefill attn+lazy-ratio TFLOP/s & % BF16 tensor peak; compaction GB/s; ratio ovh %"
+ATTN_SOURCES = ["kv_cache_compression_tcgen05_b200/csrc/attn_fwd.cuh", "kv_cache_compression_tcgen05_b200/csrc/lt_device.cuh"]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(config_name):
+    """DRAM bytes per attention launch from the committed ncu summary, or None if
+    the kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{config_name}.traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_source_sha") != source_digest(ATTN_SOURCES):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def attention_flops(cfg):
+    """Algorithmic causal FLOPs of one layer: 4 d per (query, key <= query, head)."""
+    return 4.0 * cfg.d * cfg.hq * cfg.causal_pairs()
+
+
+def ratio_flops(cfg):
+    """2 d FLOPs per (observed row, head, key in K_i)."""
+    total = 0
+    for n in cfg.seqlens:
+        nb = min(cfg.n_obs, n)
+        for i in range(n - nb, n):
+            total += min(cfg.S + cfg.W, i + 1)
+    return 2.0 * cfg.d * cfg.hq * total
+
+
+def compaction_bytes(cfg, n_layers):
+    """Bytes read + written by compacting n_layers demoted layers (K and V)."""
+    rows = sum(min(n, cfg.S + cfg.W) for n in cfg.seqlens)
+    return 2.0 * 2.0 * rows * cfg.hkv * cfg.d * 2 * n_layers
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ------------------------------------------------------------------ our arm
+
+class Prefill:
+    """The whole path over every layer of one prefill, inputs resident on the GPU."""
+
+    def __init__(self, cfg, lt, device="cuda"):
+        self.cfg, self.lt = cfg, lt
+        self.layers = [synth.layer_inputs(cfg, l, device) for l in range(cfg.layers)]
+        T, H, d = cfg.total_tokens, cfg.hq, cfg.d
+        self.cu = torch.tensor(cfg.cu_seqlens(), dtype=torch.int32, device=device) if cfg.batch > 1 else None
+        self.O = torch.empty((T, H, d), dtype=torch.bfloat16, device=device)
+        self.LSE = torch.empty((H, T), dtype=torch.float32, device=device)
+        self.ratio_dev = torch.empty((cfg.layers, cfg.batch, H), dtype=torch.float32, device=device)
+        self.ratio_host = torch.empty((cfg.layers, cfg.batch, H), dtype=torch.float32, pin_memory=True)
+        slots = cfg.S + cfg.W
+        self.ks = torch.empty((cfg.budget, cfg.batch, cfg.hkv, slots, d), dtype=torch.bfloat16, device=device)
+        self.vs = torch.empty_like(self.ks)
+        self.slen = torch.empty((cfg.budget, cfg.batch), dtype=torch.int32, device=device)
+        self.masks = torch.zeros((cfg.layers, cfg.batch), dtype=torch.uint8, device=device)
+        self.mask_host = torch.zeros((cfg.layers, cfg.batch), dtype=torch.uint8, pin_memory=True)
+        self.events = [torch.cuda.Event() for _ in range(cfg.layers)]
+        self.launches = 0
+        self.attn_events = None
+
+    def step(self, time_kernels=False):
+        cfg, lt = self.cfg, self.lt
+        kw = dict(cu_seqlens=self.cu, max_seqlen=cfg.max_seqlen)
+        queues = [lt.LayerQueue(cfg.layers, cfg.budget) for _ in range(cfg.batch)]
+        demoted = []
+        self.launches = 0
+        ev = [] if time_kernels else None
+        mask_host = self.mask_host.numpy()
+        mask_host[:] = 0
+
+        def consume(l):
+            # Host side of layer l: its ratios are in pinned memory once its event fires.
+            self.events[l].synchronize()
+            newly = []
+            for b in range(cfg.batch):
+                d = queues[b].push(l, lt.lt_layer_score(self.ratio_host[l, b].numpy()))
+                if d >= 0:
+                    newly.append((d, b))
+            for d, b in newly:
+                mask_host[d, b] = 1
+            for d in sorted(set(x for x, _ in newly)):
+                k = len(demoted)
+                self.masks[d].copy_(self.mask_host[d], non_blocking=True)
+                Q, K, V = self.layers[d]
+                lt.lt_compact_kv(K, V, self.masks[d], cfg.S, cfg.W, k_stream=self.ks[k % cfg.budget],
+                                 v_stream=self.vs[k % cfg.budget], stream_len=self.slen[k % cfg.budget], **kw)
+                self.launches += 1
+                demoted.append(d)
+
+        for l in range(cfg.layers):
+            Q, K, V = self.layers[l]
+            if ev is not None:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e2 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+            lt.lt_prefill_attn(Q, K, V, out=self.O, lse=self.LSE, **kw)
+            if ev is not None:
+                e1.record()
+            lt.lt_lazy_ratio(Q, K, self.LSE, cfg.S, cfg.W, cfg.n_obs, out=self.ratio_dev[l], **kw)
+            if ev is not None:
+                e2.record()
+                ev.append((e0, e1, e2))
+            self.launches += 2
+            self.ratio_host[l].copy_(self.ratio_dev[l], non_blocking=True)
+            self.events[l].record()
+            if l > 0:
+                consume(l - 1)
+        consume(cfg.layers - 1)
+        for q in queues:
+            q.close()
+        self.attn_events = ev
+        return demoted
+
+
+def run_ours(args, cfg, rank, world):
+    import kv_cache_compression_tcgen05_b200 as lt
+    lt.library()
+    peaks, peak_src = load_peaks()
+    pf = Prefill(cfg, lt)
+    for _ in range(args.warmup):
+        pf.step()
+    torch.cuda.synchronize()
+    barrier(world)
+
+    # Device-timed region: K whole steps.
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    attn_ms, ratio_ms = [], []
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        torch.cuda.synchronize()
+        start.record()
+        launches = 0
+        for _ in range(args.steps):
+            pf.step(time_kernels=True)
+            launches += pf.launches
+            for e0, e1, e2 in pf.attn_events:
+                attn_ms.append((e0, e1))
+                ratio_ms.append((e1, e2))
+        stop.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(stop), world) / args.steps
+    t_attn = statistics.mean(a.elapsed_time(b) for a, b in attn_ms) * 1e-3
+    t_ratio = statistics.mean(a.elapsed_time(b) for a, b in ratio_ms) * 1e-3
+
+    if args.kernels_only:
+        return {"metric": METRIC, "ms_per_step": round(ms, 4), "attn_us_per_layer": round(t_attn * 1e6, 2),
+                "ratio_us_per_layer": round(t_ratio * 1e6, 2), "gpu_launches": launches}
+
+    # Compaction timed on its own: every demoted layer of one step (inputs > L2 apart).
+    kw = dict(cu_seqlens=pf.cu, max_seqlen=cfg.max_seqlen)
+    mask1 = torch.ones(cfg.batch, dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+    c_times = []
+    for rep in range(5):
+        for l in range(cfg.budget):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            Q, K, V = pf.layers[l]
+            e0.record()
+            lt.lt_compact_kv(K, V, mask1, cfg.S, cfg.W, k_stream=pf.ks[0], v_stream=pf.vs[0], stream_len=pf.slen[0],
+                             **kw)
+            e1.record()
+            torch.cuda.synchronize()
+            if rep > 0:
+                c_times.append(e0.elapsed_time(e1) * 1e-3)
+    del flush
+    t_comp = statistics.mean(c_times)
+
+    fl_attn, fl_ratio = attention_flops(cfg), ratio_flops(cfg)
+    step_flops = cfg.layers * (fl_attn + fl_ratio)
+    value = world * step_flops / (ms * 1e-3) / 1e12
+    achieved = fl_attn / t_attn / 1e12
+    peak_sus = float(peaks["bf16_tflops_sustained"])
+    peak_burst = float(peaks["bf16_tflops"])
+    traffic = recorded_traffic(cfg.name)
+    comp_gbs = compaction_bytes(cfg, 1) / t_comp / 1e9
+
+    e2e = measure_e2e(args, cfg, lt, pf, world)
+    cpu = cpu_baseline(cfg) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V with per-layer sink bias; pages' datasets/weights absent)",
+        "config": {
+            "workload": f"{cfg.name}: {cfg.layers} layers, batch {cfg.batch}, seq {cfg.max_seqlen}, "
+                        f"{cfg.hq} q heads / {cfg.hkv} KV heads, head_dim {cfg.d}, S={cfg.S}, W={cfg.W}, "
+                        f"n_obs={cfg.n_obs}, budget {cfg.budget}",
+            "layers": cfg.layers, "batch": cfg.batch, "seq_len": cfg.max_seqlen, "hq": cfg.hq, "hkv": cfg.hkv,
+            "head_dim": cfg.d, "S": cfg.S, "W": cfg.W, "n_obs": cfg.n_obs, "budget": cfg.budget,
+            "l2": "inputs of one step (all layers' Q/K/V) exceed L2; no flush between steps",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "attn_tflops": round(achieved, 2),
+        "attn_pct_of_burst_peak": round(100 * achieved / peak_burst, 2),
+        "attn_us_per_layer": round(t_attn * 1e6, 2),
+        "ratio_us_per_layer": round(t_ratio * 1e6, 2),
+        "ratio_overhead_pct": round(100 * t_ratio / t_attn, 3),
+        "compaction_gbs": round(comp_gbs, 1),
+        "compaction_us_per_layer": round(t_comp * 1e6, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_sus, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak_sus, 4), "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)"},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+    }
+    return line
+
+
+def measure_e2e(args, cfg, lt, pf, world):
+    """Same metric through the public calls with host buffers: every step copies
+    each layer's Q/K/V from pinned host memory to the device and reads back each
+    layer's O and LSE, the ratios and the compacted KV, all inside the
+    device-timed region.  Uploads run on a side stream one layer ahead, read-backs
+    on another, so copies overlap the kernels.  The full K/V of every layer stay
+    on the device (the KV cache the queue manages); Q is double buffered."""
+    host = [tuple(t.cpu().pin_memory() for t in lay) for lay in pf.layers]
+    T, H, d = cfg.total_tokens, cfg.hq, cfg.d
+    dev_q = [torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    dev_kv = [tuple(torch.empty_like(t) for t in lay[1:]) for lay in pf.layers]
+    o_host = torch.empty((cfg.layers, T, H, d), dtype=torch.bfloat16, pin_memory=True)
+    lse_host = torch.empty((cfg.layers, H, T), dtype=torch.float32, pin_memory=True)
+    ks_host = torch.empty(pf.ks.shape, dtype=torch.bfloat16, pin_memory=True)
+    vs_host = torch.empty_like(ks_host)
+    O = [torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    LSE = [torch.empty((H, T), dtype=torch.float32, device="cuda") for _ in range(2)]
+    copy_in, copy_out = torch.cuda.Stream(), torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+    kw = dict(cu_seqlens=pf.cu, max_seqlen=cfg.max_seqlen)
+    h2d = sum(t.numel() * t.element_size() for lay in host for t in lay)
+    d2h = (o_host.numel() * 2 + lse_host.numel() * 4 + pf.ratio_host.numel() * 4 + 2 * ks_host.numel() * 2)
+
+    def one_step():
+        ready = [torch.cuda.Event() for _ in range(cfg.layers)]
+        done = [torch.cuda.Event() for _ in range(cfg.layers)]
+        queues = [lt.LayerQueue(cfg.layers, cfg.budget) for _ in range(cfg.batch)]
+        n_dem = 0
+        mask_host = pf.mask_host.numpy()
+
+        def upload(l):
+            with torch.cuda.stream(copy_in):
+                if l >= 2:
+                    copy_in.wait_event(done[l - 2])   # Q buffer and O/LSE of layer l-2 consumed
+                dev_q[l % 2].copy_(host[l][0], non_blocking=True)
+                dev_kv[l][0].copy_(host[l][1], non_blocking=True)
+                dev_kv[l][1].copy_(host[l][2], non_blocking=True)
+                ready[l].record(copy_in)
+
+        upload(0)
+        for l in range(cfg.layers):
+            if l + 1 < cfg.layers:
+                upload(l + 1)
+            main.wait_event(ready[l])
+            Q, (K, V) = dev_q[l % 2], dev_kv[l]
+            lt.lt_prefill_attn(Q, K, V, out=O[l % 2], lse=LSE[l % 2], **kw)
+            lt.lt_lazy_ratio(Q, K, LSE[l % 2], cfg.S, cfg.W, cfg.n_obs, out=pf.ratio_dev[l], **kw)
+            pf.ratio_host[l].copy_(pf.ratio_dev[l], non_blocking=True)
+            pf.events[l].record()
+            with torch.cuda.stream(copy_out):
+                copy_out.wait_event(pf.events[l])
+                o_host[l].copy_(O[l % 2], non_blocking=True)
+                lse_host[l].copy_(LSE[l % 2], non_blocking=True)
+                done[l].record(copy_out)
+            pf.events[l].synchronize()
+            mask_host[l] = 0
+            dem = []
+            for b in range(cfg.batch):
+                m = queues[b].push(l, lt.lt_layer_score(pf.ratio_host[l, b].numpy()))
+                if m >= 0:
+                    dem.append((m, b))
+            for m in sorted(set(x for x, _ in dem)):
+                mask_host[m] = 0
+                for x, b in dem:
+                    if x == m:
+                        mask_host[m, b] = 1
+                pf.masks[m].copy_(pf.mask_host[m], non_blocking=True)
+                lt.lt_compact_kv(dev_kv[m][0], dev_kv[m][1], pf.masks[m], cfg.S, cfg.W,
+                                 k_stream=pf.ks[n_dem % cfg.budget], v_stream=pf.vs[n_dem % cfg.budget],
+                                 stream_len=pf.slen[n_dem % cfg.budget], **kw)
+                n_dem += 1
+        with torch.cuda.stream(copy_out):
+            copy_out.wait_stream(main)
+            ks_host.copy_(pf.ks, non_blocking=True)
+            vs_host.copy_(pf.vs, non_blocking=True)
+        main.wait_stream(copy_out)
+        main.wait_stream(copy_in)
+        for q in queues:
+            q.close()
+
+    for _ in range(2):
+        one_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(1, min(args.steps, 5))
+    e0.record()
+    for _ in range(steps):
+        one_step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    step_flops = cfg.layers * (attention_flops(cfg) + ratio_flops(cfg))
+    return {"value": round(world * step_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 3)}
+
+
+# ------------------------------------------------------------- CPU (oracle)
+
+def oracle_sample(cfg, seconds, seed=0):
+    """Time the fp64 oracle on a bounded random sample of the workload's rows:
+    attention rows (uniform over tokens and heads) of layer 0 plus the lazy
+    ratio of a proportional share of the observed rows.  Returns
+    (TFLOP/s, cores, description)."""
+    import oracle
+    Q, K, V = synth.layer_inputs(cfg, 0, "cpu")
+    q, k, v = synth.bf16_bits(Q), synth.bf16_bits(K), synth.bf16_bits(V)
+    cu = np.array(cfg.cu_seqlens(), np.int32)
+    cores = os.cpu_count() or 1
+    rng = np.random.default_rng(seed)
+    starts = np.array(cfg.cu_seqlens()[:-1])
+
+    def run(n):
+        toks = rng.integers(0, cfg.total_tokens, n).astype(np.int32)
+        heads = rng.integers(0, cfg.hq, n).astype(np.int32)
+        pos = toks - starts[np.searchsorted(starts, toks, side="right") - 1]
+        t0 = time.perf_counter()
+        oracle.attn(cu, q, k, v, tokens=toks, heads=heads, nthreads=cores)
+        t = time.perf_counter() - t0
+        return 4.0 * cfg.d * float(np.sum(pos + 1)), t
+
+    fl, t = run(64)
+    n = int(min(200000, max(64, 64 * seconds / max(t, 1e-3))))
+    fl, t = run(n)
+    return fl / t / 1e12, cores, f"{n} random (token, head) attention rows of layer 0 ({fl / 1e9:.1f} GFLOP, {t:.1f} s)"
+
+
+def cpu_baseline(cfg, seconds=10.0):
+    v, cores, desc = oracle_sample(cfg, seconds)
+    return {"value": round(v, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+
+
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return None
+    vals = []
+    desc = ""
+    for _ in range(args.warmup):
+        oracle_sample(cfg, 2.0, seed=1)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        v, cores, desc = oracle_sample(cfg, 5.0, seed=100 + s)
+        vals.append(v)
+    ms = (time.perf_counter() - t0) * 1e3 / max(1, args.steps)
+    value = statistics.mean(vals)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.name} (fp64 CPU oracle on a bounded random row sample per step)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="gqa1p2b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernels-only", action="store_true",
+                    help="time only the device steps (no e2e, CPU baseline or compaction leg); for profiling")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    cfg = synth.CONFIGS[args.config]
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, cfg, rank, args.gpus)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    rank, world, _ = dist_setup(args.gpus)
+    line = run_ours(args, cfg, rank, world)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,186 @@
+/*
+ * lt.h -- C ABI of the LightTransfer-Test prefill hot path on B200 (sm_100a).
+ *
+ * LightTransfer-Test converts "lazy" layers of a dense transformer to streaming
+ * attention on the fly, from the prefill alone.  The path has four steps:
+ *
+ *   1. lt_prefill_attn  causal GQA prefill attention that also writes the per-row
+ *                       log-sum-exp (LSE) of the attention logits;
+ *   2. lt_lazy_ratio    the lazy ratio of each (sequence, query head), computed
+ *                       with that LSE as its denominator so that only the S sink
+ *                       and W recent keys of each observed query are visited;
+ *   3. lt_select_layers / lt_queue_*  the layer priority queue that demotes the
+ *                       layer with the highest ratio once more than the allowed
+ *                       number of full-KV layers are queued;
+ *   4. lt_compact_kv    the gather that keeps a demoted layer's sink and recent
+ *                       rows as its streaming KV cache.
+ *
+ * Sources (the LightTransfer pages):
+ *   - LightTransfer write-up (xzbcqc.com news page), the two problems of
+ *     LightTransfer-Test and their solutions: FlashAttention does not store the
+ *     attention weights, so the LSE it produces is used as the ratio's
+ *     denominator and the numerator costs O(1) per query instead of O(seq_len);
+ *     a priority queue keyed by lazy ratio keeps the prefill's peak memory at
+ *     most 50% full KV + 50% streaming KV.
+ *   - Press-release page "LLM突破：推理加速，长CoT生成惊艳", section
+ *     "LightTransfer方法详解": the lazy ratio is the sum of the attention weights
+ *     from the query to the initial and the recent keys.
+ *   - LightTransfer project page, Methodology / LightTransfer-Test, Figure 2
+ *     caption: after each layer the ratio and layer index enter the queue; once
+ *     it is full the layer with the highest ratio is made lazy and its KV cache
+ *     reduced, freeing memory for the current layer.
+ *
+ * Conventions for every call:
+ *   - Tensor pointers marked "device" are caller-owned CUDA device memory; the
+ *     library never allocates, frees or keeps them.  Tensors are row-major and
+ *     contiguous; bf16 tensors are passed as void*; every device pointer must be
+ *     16-byte aligned.  When total_tokens is 0 the token-indexed inputs and
+ *     outputs (Q, K, V, O, LSE) are not accessed and may be null.
+ *   - Calls that take a stream only enqueue work on it (they never synchronise
+ *     the device); their outputs are ready when the stream reaches them.
+ *   - Arguments are checked before anything is enqueued.  A failed check returns
+ *     LT_ERR_INVALID_ARG (or LT_ERR_UNSUPPORTED for a head_dim other than 64 or
+ *     128) and enqueues nothing.  A launch failure returns LT_ERR_CUDA.
+ *   - Kernels never wait unboundedly: a wait that exceeds its limit sets a
+ *     device status word and the kernel returns early; lt_device_status reports
+ *     it as LT_ERR_TIMEOUT.
+ */
+#ifndef LT_H_
+#define LT_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LT_OK = 0,
+  LT_ERR_INVALID_ARG = 1, /* a pointer, size or layout is invalid */
+  LT_ERR_UNSUPPORTED = 2, /* valid but not implemented (head_dim not 64/128) */
+  LT_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  LT_ERR_TIMEOUT = 4      /* a kernel gave up a bounded wait (see lt_device_status) */
+} lt_status;
+
+/* A cudaStream_t (the runtime's stream handle); NULL is the legacy default stream. */
+typedef struct CUstream_st* lt_stream;
+
+/*
+ * Shape of one packed prefill batch.
+ *   batch        number of sequences (>= 1)
+ *   total_tokens T = sum of the sequence lengths (>= 0)
+ *   max_seqlen   the longest sequence length; every sequence must be at most
+ *                this long (tiles beyond it are never scheduled)
+ *   hq, hkv      query heads and key/value heads; hq % hkv == 0, query head h
+ *                reads KV head h / (hq / hkv)
+ *   head_dim     d, 64 or 128
+ *   cu_seqlens   device int32 [batch + 1]: sequence b is tokens
+ *                [cu_seqlens[b], cu_seqlens[b+1]); NULL means batch == 1 and one
+ *                sequence of total_tokens tokens.
+ */
+typedef struct {
+  int batch;
+  int total_tokens;
+  int max_seqlen;
+  int hq;
+  int hkv;
+  int head_dim;
+  const int32_t* cu_seqlens;
+} lt_shape;
+
+/*
+ * Causal GQA prefill attention with the per-row LSE.
+ *   For sequence b, query row i (position inside b), query head h, KV head
+ *   kh = h / (hq/hkv):  s_ij = scale * q_i . k_j for j <= i (same sequence),
+ *   LSE_i = log sum_j exp(s_ij),  O_i = sum_j exp(s_ij - LSE_i) v_j.
+ * Q: device bf16 [T, hq, d]; K, V: device bf16 [T, hkv, d].
+ * O: device bf16 [T, hq, d] (written); LSE: device fp32 [hq, T] (natural log,
+ * written).  softmax_scale <= 0 selects 1/sqrt(d).
+ * Source: the write-up's first solution (FlashAttention's LSE as the ratio's
+ * denominator); the attention itself is plain causal softmax attention.
+ */
+lt_status lt_prefill_attn(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
+                          float* LSE, float softmax_scale, lt_stream stream);
+
+/*
+ * Lazy ratio from the LSE.
+ *   For every sequence b (length N), query head h and each of the last
+ *   n' = min(n_obs, N) rows i of b:
+ *     K_i = [0, min(S, i+1))  U  [max(S, i-W+1), i]      (sink + recent keys)
+ *     r_i = sum_{j in K_i} exp(scale * q_i . k_j - LSE_i)
+ *   ratio[b, h] = mean of r_i over those rows (0 when N == 0).
+ * Q, K as for lt_prefill_attn; LSE: device fp32 [hq, T] as written by it.
+ * ratio: device fp32 [batch, hq] (written).  S >= 0, W >= 0, S + W >= 1,
+ * 1 <= n_obs <= 4096.
+ * Sources: the press-release page's definition (attention weights to the
+ * initial and recent keys) and the write-up's first solution (LSE as the
+ * denominator; O(S+W) work per query).
+ */
+lt_status lt_lazy_ratio(const lt_shape* shape, const void* Q, const void* K, const float* LSE,
+                        float softmax_scale, int S, int W, int n_obs, float* ratio, lt_stream stream);
+
+/* Score of one layer of one sequence: the mean of its hq ratios (host). */
+float lt_layer_score(const float* ratio_of_heads, int hq);
+
+/*
+ * Offline selection (every layer's ratio known; the post-prefill route the
+ * write-up contrasts the queue with).  ratios: host fp32 [L, batch, hq].  For each
+ * sequence the layers are ranked by (score descending, layer ascending) and
+ * the first `budget` are lazy.  lazy_mask: host uint8 [batch, L] (written, 0/1);
+ * order: host int32 [batch, budget] (nullable; written in rank order).
+ * 0 <= budget <= L.  Scores that are NaN are rejected.  Host-only, synchronous.
+ */
+lt_status lt_select_layers(const float* ratios, int L, int batch, int hq, int budget, uint8_t* lazy_mask,
+                           int32_t* order);
+
+/*
+ * Online layer priority queue of one sequence (project page, Figure 2 caption;
+ * write-up, second solution).  Capacity C = L - budget full-KV layers.
+ * lt_queue_push adds (layer, score); if more than C layers are then queued, the
+ * best-ranked one (highest score; lower index on a tie) is popped and returned
+ * in *demoted (else -1): that layer becomes a streaming layer.  Pushing each
+ * of the L layers once demotes exactly `budget` layers, the same set as
+ * lt_select_layers.  A layer pushed twice, out of range, or with a non-finite
+ * score is rejected with LT_ERR_INVALID_ARG and leaves the queue unchanged.
+ * Host-only, synchronous; one queue per sequence; not thread-safe.
+ */
+typedef struct lt_queue lt_queue;
+lt_status lt_queue_create(int L, int budget, lt_queue** queue);
+lt_status lt_queue_push(lt_queue* queue, int layer, float score, int* demoted);
+int lt_queue_size(const lt_queue* queue);
+void lt_queue_destroy(lt_queue* queue);
+
+/*
+ * KV-cache compaction of one layer to its streaming version.
+ *   For every sequence b with mask[b] != 0 (length N):
+ *     p = [0, min(S, N)) ++ [max(S, N - W), N)      (kept positions, in order)
+ *     K_stream[b, kh, r, :] = K[cu[b] + p_r, kh, :]  for r < len = |p| = min(N, S+W)
+ *     rows r >= len are zero; stream_len[b] = len.  Same for V.
+ *   Sequences with mask[b] == 0 are not touched and get stream_len[b] = 0.
+ * K, V: device bf16 [T, hkv, d]; mask: device uint8 [batch];
+ * K_stream, V_stream: device bf16 [batch, hkv, S + W, d]; stream_len: device
+ * int32 [batch].  S >= 0, W >= 0, S + W >= 1.  After this call is enqueued the
+ * caller may release the layer's full K/V in stream order (the write-up's
+ * "switch its KV cache to the streaming version").
+ */
+lt_status lt_compact_kv(const lt_shape* shape, const void* K, const void* V, const uint8_t* mask, int S, int W,
+                        void* K_stream, void* V_stream, int32_t* stream_len, lt_stream stream);
+
+/*
+ * Device status word of the current device: LT_OK, or LT_ERR_TIMEOUT if a kernel
+ * gave up a bounded wait since the last clear.  Synchronises the device.
+ * clear != 0 resets the word.
+ */
+lt_status lt_device_status(int clear);
+
+/* Human-readable name of a status. */
+const char* lt_status_string(lt_status status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int lt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LT_H_ */

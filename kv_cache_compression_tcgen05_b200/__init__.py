@@ -1,0 +1,36 @@
+"""LightTransfer-Test prefill hot path on B200 (sm_100a).
+
+A thin Python binding over the C ABI of ``liblt.so`` (declared in
+``include/lt.h``).  Every function keeps the C name and only marshals
+arguments: it checks tensor dtypes/devices/shapes, allocates outputs with
+PyTorch when the caller passes none, and calls the library on the current CUDA
+stream.  All arithmetic runs in the library's CUDA kernels; if the library is
+missing the calls raise instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+from .binding import (  # noqa: F401
+    LT_ERR_CUDA,
+    LT_ERR_INVALID_ARG,
+    LT_ERR_TIMEOUT,
+    LT_ERR_UNSUPPORTED,
+    LT_OK,
+    LtError,
+    LtShape,
+    library,
+    library_path,
+    lt_compact_kv,
+    lt_device_status,
+    lt_layer_score,
+    lt_lazy_ratio,
+    lt_prefill_attn,
+    lt_queue_create,
+    lt_queue_destroy,
+    lt_queue_push,
+    lt_queue_size,
+    lt_select_layers,
+    lt_status_string,
+    lt_version,
+    LayerQueue,
+)
+from .build import build  # noqa: F401

@@ -1,0 +1,284 @@
+"""ctypes binding of ``liblt.so``: the C functions of ``include/lt.h`` under the
+same names, with torch tensors in and out.  Argument marshalling only."""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+import torch
+
+from .build import LIB
+
+LT_OK = 0
+LT_ERR_INVALID_ARG = 1
+LT_ERR_UNSUPPORTED = 2
+LT_ERR_CUDA = 3
+LT_ERR_TIMEOUT = 4
+
+_lock = threading.Lock()
+_lib = None
+
+
+class LtShape(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int),
+        ("total_tokens", ctypes.c_int),
+        ("max_seqlen", ctypes.c_int),
+        ("hq", ctypes.c_int),
+        ("hkv", ctypes.c_int),
+        ("head_dim", ctypes.c_int),
+        ("cu_seqlens", ctypes.c_void_p),
+    ]
+
+
+class LtError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {lt_status_string(status)}")
+        self.status = status
+
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+_shp = ctypes.POINTER(LtShape)
+
+_SIGS = {
+    "lt_prefill_attn": (_i, [_shp, _vp, _vp, _vp, _vp, _vp, _f, _vp]),
+    "lt_lazy_ratio": (_i, [_shp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
+    "lt_layer_score": (_f, [_vp, _i]),
+    "lt_select_layers": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
+    "lt_queue_create": (_i, [_i, _i, ctypes.POINTER(_vp)]),
+    "lt_queue_push": (_i, [_vp, _i, _f, ctypes.POINTER(_i)]),
+    "lt_queue_size": (_i, [_vp]),
+    "lt_queue_destroy": (None, [_vp]),
+    "lt_compact_kv": (_i, [_shp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp]),
+    "lt_device_status": (_i, [_i]),
+    "lt_status_string": (ctypes.c_char_p, [_i]),
+    "lt_version": (_i, []),
+}
+
+
+def library_path() -> str:
+    return LIB
+
+
+def library():
+    """The loaded ``liblt.so``; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB):
+                raise RuntimeError(f"{LIB} is missing: build it with "
+                                   "`python -m kv_cache_compression_tcgen05_b200.build`")
+            lib = ctypes.CDLL(LIB)
+            for name, (res, args) in _SIGS.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def lt_status_string(status: int) -> str:
+    return library().lt_status_string(int(status)).decode()
+
+
+def lt_version() -> int:
+    return library().lt_version()
+
+
+def _check(status: int, where: str):
+    if status != LT_OK:
+        raise LtError(status, where)
+
+
+def _stream_handle(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _dev_tensor(t, name, dtype, ndim=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _shape(T, hq, hkv, d, cu_seqlens, max_seqlen):
+    s = LtShape()
+    s.total_tokens = int(T)
+    s.hq = int(hq)
+    s.hkv = int(hkv)
+    s.head_dim = int(d)
+    if cu_seqlens is None:
+        s.batch = 1
+        s.max_seqlen = int(T)
+        s.cu_seqlens = None
+    else:
+        _dev_tensor(cu_seqlens, "cu_seqlens", torch.int32, 1)
+        s.batch = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        s.max_seqlen = int(max_seqlen)
+        s.cu_seqlens = cu_seqlens.data_ptr()
+    return s
+
+
+def lt_prefill_attn(Q, K, V, cu_seqlens=None, max_seqlen=None, softmax_scale=None, out=None, lse=None,
+                    stream=None):
+    """Causal GQA prefill attention.  Q [T, hq, d], K/V [T, hkv, d] bf16 (CUDA).
+    Returns (O [T, hq, d] bf16, LSE [hq, T] fp32)."""
+    _dev_tensor(Q, "Q", torch.bfloat16, 3)
+    _dev_tensor(K, "K", torch.bfloat16, 3)
+    _dev_tensor(V, "V", torch.bfloat16, 3)
+    T, hq, d = Q.shape
+    hkv = K.shape[1]
+    if K.shape != (T, hkv, d) or V.shape != K.shape:
+        raise ValueError("K and V must be [T, hkv, d] with Q's T and d")
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty((hq, T), dtype=torch.float32, device=Q.device)
+    _dev_tensor(out, "out", torch.bfloat16, 3)
+    _dev_tensor(lse, "lse", torch.float32, 2)
+    if out.shape != Q.shape or lse.shape != (hq, T):
+        raise ValueError("out must be [T, hq, d] and lse [hq, T]")
+    shape = _shape(T, hq, hkv, d, cu_seqlens, max_seqlen)
+    _check(library().lt_prefill_attn(ctypes.byref(shape), Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                     out.data_ptr(), lse.data_ptr(),
+                                     0.0 if softmax_scale is None else float(softmax_scale),
+                                     _stream_handle(stream)), "lt_prefill_attn")
+    return out, lse
+
+
+def lt_lazy_ratio(Q, K, LSE, S, W, n_obs, cu_seqlens=None, max_seqlen=None, softmax_scale=None, out=None,
+                  stream=None):
+    """Lazy ratio [batch, hq] fp32 from Q, K and the attention's LSE [hq, T]."""
+    _dev_tensor(Q, "Q", torch.bfloat16, 3)
+    _dev_tensor(K, "K", torch.bfloat16, 3)
+    _dev_tensor(LSE, "LSE", torch.float32, 2)
+    T, hq, d = Q.shape
+    hkv = K.shape[1]
+    if K.shape != (T, hkv, d) or LSE.shape != (hq, T):
+        raise ValueError("K must be [T, hkv, d] and LSE [hq, T]")
+    shape = _shape(T, hq, hkv, d, cu_seqlens, max_seqlen)
+    if out is None:
+        out = torch.empty((shape.batch, hq), dtype=torch.float32, device=Q.device)
+    _dev_tensor(out, "out", torch.float32, 2)
+    if out.shape != (shape.batch, hq):
+        raise ValueError("out must be [batch, hq]")
+    _check(library().lt_lazy_ratio(ctypes.byref(shape), Q.data_ptr(), K.data_ptr(), LSE.data_ptr(),
+                                   0.0 if softmax_scale is None else float(softmax_scale), int(S), int(W),
+                                   int(n_obs), out.data_ptr(), _stream_handle(stream)), "lt_lazy_ratio")
+    return out
+
+
+def lt_compact_kv(K, V, mask, S, W, cu_seqlens=None, max_seqlen=None, k_stream=None, v_stream=None,
+                  stream_len=None, stream=None):
+    """Streaming KV of the sequences with mask[b] != 0.
+    Returns (K_stream, V_stream [batch, hkv, S+W, d] bf16, stream_len [batch] int32)."""
+    _dev_tensor(K, "K", torch.bfloat16, 3)
+    _dev_tensor(V, "V", torch.bfloat16, 3)
+    _dev_tensor(mask, "mask", torch.uint8, 1)
+    T, hkv, d = K.shape
+    if V.shape != K.shape:
+        raise ValueError("V must match K")
+    shape = _shape(T, hkv, hkv, d, cu_seqlens, max_seqlen)
+    if mask.numel() != shape.batch:
+        raise ValueError("mask must have one entry per sequence")
+    slots = int(S) + int(W)
+    if k_stream is None:
+        k_stream = torch.empty((shape.batch, hkv, slots, d), dtype=torch.bfloat16, device=K.device)
+    if v_stream is None:
+        v_stream = torch.empty((shape.batch, hkv, slots, d), dtype=torch.bfloat16, device=K.device)
+    if stream_len is None:
+        stream_len = torch.empty((shape.batch,), dtype=torch.int32, device=K.device)
+    for t, n in ((k_stream, "k_stream"), (v_stream, "v_stream")):
+        _dev_tensor(t, n, torch.bfloat16, 4)
+        if t.shape != (shape.batch, hkv, slots, d):
+            raise ValueError(f"{n} must be [batch, hkv, S+W, d]")
+    _dev_tensor(stream_len, "stream_len", torch.int32, 1)
+    _check(library().lt_compact_kv(ctypes.byref(shape), K.data_ptr(), V.data_ptr(), mask.data_ptr(), int(S),
+                                   int(W), k_stream.data_ptr(), v_stream.data_ptr(), stream_len.data_ptr(),
+                                   _stream_handle(stream)), "lt_compact_kv")
+    return k_stream, v_stream, stream_len
+
+
+def _host_f32(x):
+    a = x.detach().cpu().numpy() if isinstance(x, torch.Tensor) else np.asarray(x)
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def lt_layer_score(ratio_of_heads) -> float:
+    r = _host_f32(ratio_of_heads).ravel()
+    return float(library().lt_layer_score(r.ctypes.data, r.size))
+
+
+def lt_select_layers(ratios, budget):
+    """Offline selection.  ratios [L, batch, hq] (host); returns
+    (lazy_mask [batch, L] uint8, order [batch, budget] int32) as numpy arrays."""
+    r = _host_f32(ratios)
+    if r.ndim != 3:
+        raise ValueError("ratios must be [L, batch, hq]")
+    L, B, H = r.shape
+    lazy = np.empty((B, L), np.uint8)
+    order = np.empty((B, max(int(budget), 1)), np.int32)
+    _check(library().lt_select_layers(r.ctypes.data, L, B, H, int(budget), lazy.ctypes.data, order.ctypes.data),
+           "lt_select_layers")
+    return lazy, order[:, : int(budget)]
+
+
+def lt_queue_create(L, budget):
+    q = ctypes.c_void_p()
+    _check(library().lt_queue_create(int(L), int(budget), ctypes.byref(q)), "lt_queue_create")
+    return q
+
+
+def lt_queue_push(q, layer, score) -> int:
+    demoted = ctypes.c_int(-1)
+    _check(library().lt_queue_push(q, int(layer), float(score), ctypes.byref(demoted)), "lt_queue_push")
+    return demoted.value
+
+
+def lt_queue_size(q) -> int:
+    return library().lt_queue_size(q)
+
+
+def lt_queue_destroy(q):
+    library().lt_queue_destroy(q)
+
+
+class LayerQueue:
+    """Owning wrapper of one lt_queue (one sequence)."""
+
+    def __init__(self, L, budget):
+        self._q = lt_queue_create(L, budget)
+
+    def push(self, layer, score) -> int:
+        return lt_queue_push(self._q, layer, score)
+
+    def __len__(self):
+        return lt_queue_size(self._q)
+
+    def close(self):
+        if self._q is not None:
+            lt_queue_destroy(self._q)
+            self._q = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def lt_device_status(clear: bool = True) -> int:
+    """LT_OK or LT_ERR_TIMEOUT (synchronises the current device)."""
+    return library().lt_device_status(1 if clear else 0)

@@ -1,0 +1,255 @@
+// lt_api.cu -- the device entry points of the C ABI declared in include/lt.h:
+// argument checks, TMA descriptors and kernel launches.  Nothing here
+// allocates device memory or synchronises (except lt_device_status).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <mutex>
+
+#include "attn_fwd.cuh"
+#include "compact_kv.cuh"
+#include "lazy_ratio.cuh"
+#include "lt.h"
+
+namespace {
+
+// Device status word: bit lt::kErrTimeout is set by a kernel that gave up a
+// bounded wait.  One copy per device; read and cleared by lt_device_status.
+__device__ unsigned g_status_word;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sm_count = 0;
+  unsigned* status = nullptr;  // device address of g_status_word
+};
+
+std::mutex g_mutex;
+DeviceInfo g_devices[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Per-device set-up, once, with the device current.
+lt_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LT_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& info = g_devices[dev];
+  if (!info.ready) {
+    if (cudaDeviceGetAttribute(&info.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return LT_ERR_CUDA;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess) return LT_ERR_CUDA;
+    info.status = static_cast<unsigned*>(addr);
+    if (cudaFuncSetAttribute(lt::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             lt::AttnLayout<64>::kAlloc) != cudaSuccess ||
+        cudaFuncSetAttribute(lt::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             lt::AttnLayout<128>::kAlloc) != cudaSuccess ||
+        cudaFuncSetAttribute(lt::lazy_ratio_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             lt::RatioLayout<64>::bytes(lt::kRatioMaxGroup * 256)) != cudaSuccess ||
+        cudaFuncSetAttribute(lt::lazy_ratio_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             lt::RatioLayout<128>::bytes(lt::kRatioMaxGroup * 256)) != cudaSuccess)
+      return LT_ERR_CUDA;
+    info.ready = true;
+  }
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return LT_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  *out = &info;
+  return LT_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return p && (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Common checks of a packed-batch shape.
+lt_status check_shape(const lt_shape* s) {
+  if (!s) return LT_ERR_INVALID_ARG;
+  if (s->batch < 1 || s->total_tokens < 0 || s->max_seqlen < 0 || s->hq < 1 || s->hkv < 1) return LT_ERR_INVALID_ARG;
+  if (s->hq % s->hkv != 0) return LT_ERR_INVALID_ARG;
+  if (!s->cu_seqlens && s->batch != 1) return LT_ERR_INVALID_ARG;
+  if (s->cu_seqlens && !aligned(s->cu_seqlens, 4)) return LT_ERR_INVALID_ARG;
+  if (s->head_dim != 64 && s->head_dim != 128) return LT_ERR_UNSUPPORTED;
+  // Element offsets are computed in 64 bits, but token indices are int.
+  if ((long long)s->total_tokens * s->hq * s->head_dim > (1LL << 40)) return LT_ERR_INVALID_ARG;
+  return LT_OK;
+}
+
+// 3-D tensor map over a [T, heads, d] bf16 tensor: box of 128 rows x 64 columns
+// of one head, 128-byte swizzle (the layout the MMA descriptors expect).
+lt_status make_map(CUtensorMap* map, const void* base, int d, int heads, int T) {
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(heads), cuuint64_t(T)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(heads) * d * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                        estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LT_OK : LT_ERR_CUDA;
+}
+
+float resolve_scale(float softmax_scale, int d) {
+  return softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(d));
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace
+
+extern "C" {
+
+lt_status lt_prefill_attn(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O, float* LSE,
+                          float softmax_scale, lt_stream stream) {
+  lt_status st = check_shape(shape);
+  if (st != LT_OK) return st;
+  if (!std::isfinite(softmax_scale)) return LT_ERR_INVALID_ARG;
+  const int T = shape->total_tokens;
+  const int max_len = shape->cu_seqlens ? shape->max_seqlen : T;
+  if (T == 0) return LT_OK;  // nothing to read or write; the pointers may be null
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || !aligned(LSE, 4))
+    return LT_ERR_INVALID_ARG;
+  if (max_len == 0) return LT_OK;
+  const long long n_qtiles = (max_len + 127) / 128;
+  const long long num_tiles = n_qtiles * shape->batch * shape->hq;
+  if (num_tiles > INT_MAX) return LT_ERR_INVALID_ARG;
+
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != LT_OK) return st;
+  const int d = shape->head_dim;
+  CUtensorMap mq, mk, mv;
+  if (make_map(&mq, Q, d, shape->hq, T) != LT_OK || make_map(&mk, K, d, shape->hkv, T) != LT_OK ||
+      make_map(&mv, V, d, shape->hkv, T) != LT_OK)
+    return LT_ERR_INVALID_ARG;
+
+  lt::AttnParams p;
+  p.batch = shape->batch;
+  p.total_tokens = T;
+  p.hq = shape->hq;
+  p.hkv = shape->hkv;
+  p.n_qtiles = int(n_qtiles);
+  p.num_tiles = int(num_tiles);
+  p.cu_seqlens = shape->cu_seqlens;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.LSE = LSE;
+  p.scale_log2 = resolve_scale(softmax_scale, d) * kLog2e;
+  p.status = dev->status;
+  const int grid = int(num_tiles < dev->sm_count ? num_tiles : dev->sm_count);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    lt::attn_fwd_kernel<64><<<grid, lt::AttnLayout<64>::kThreads, lt::AttnLayout<64>::kAlloc, s>>>(mq, mk, mv, p);
+  else
+    lt::attn_fwd_kernel<128><<<grid, lt::AttnLayout<128>::kThreads, lt::AttnLayout<128>::kAlloc, s>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_lazy_ratio(const lt_shape* shape, const void* Q, const void* K, const float* LSE, float softmax_scale,
+                        int S, int W, int n_obs, float* ratio, lt_stream stream) {
+  lt_status st = check_shape(shape);
+  if (st != LT_OK) return st;
+  // With no tokens only `ratio` is written (zeros); the inputs may be null.
+  if (!aligned(ratio, 4)) return LT_ERR_INVALID_ARG;
+  if (shape->total_tokens > 0 && (!aligned(Q, 16) || !aligned(K, 16) || !aligned(LSE, 4))) return LT_ERR_INVALID_ARG;
+  if (S < 0 || W < 0 || (long long)S + W < 1 || n_obs < 1 || n_obs > 4096) return LT_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return LT_ERR_INVALID_ARG;
+  const int group = shape->hq / shape->hkv;
+  if (group > lt::kRatioMaxGroup) return LT_ERR_UNSUPPORTED;
+
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != LT_OK) return st;
+  lt::RatioParams p;
+  p.batch = shape->batch;
+  p.total_tokens = shape->total_tokens;
+  p.hq = shape->hq;
+  p.hkv = shape->hkv;
+  p.group = group;
+  p.S = S;
+  p.W = W;
+  p.n_obs = n_obs;
+  p.cu_seqlens = shape->cu_seqlens;
+  p.Q = static_cast<const __nv_bfloat16*>(Q);
+  p.K = static_cast<const __nv_bfloat16*>(K);
+  p.LSE = LSE;
+  p.scale_log2 = resolve_scale(softmax_scale, shape->head_dim) * kLog2e;
+  p.ratio = ratio;
+
+  // Cluster size: enough CTAs that each stages about 64 or more keys of the band.
+  const long long max_len = shape->cu_seqlens ? shape->max_seqlen : shape->total_tokens;
+  const long long band = std::min<long long>(S, max_len) + std::min<long long>(max_len, (long long)n_obs + W - 1);
+  int cluster = int(std::min<long long>(lt::kRatioMaxCluster, std::max<long long>(1, (band + 63) / 64)));
+  p.n_units = group * ((n_obs + 15) / 16);
+  const int warps = std::max(4, std::min(lt::kRatioMaxWarps, p.n_units));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cluster, shape->hkv, shape->batch);
+  cfg.blockDim = dim3(32 * warps, 1, 1);
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (shape->head_dim == 64) {
+    cfg.dynamicSmemBytes = lt::RatioLayout<64>::bytes(p.n_units);
+    e = cudaLaunchKernelEx(&cfg, lt::lazy_ratio_kernel<64>, p);
+  } else {
+    cfg.dynamicSmemBytes = lt::RatioLayout<128>::bytes(p.n_units);
+    e = cudaLaunchKernelEx(&cfg, lt::lazy_ratio_kernel<128>, p);
+  }
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_compact_kv(const lt_shape* shape, const void* K, const void* V, const uint8_t* mask, int S, int W,
+                        void* K_stream, void* V_stream, int32_t* stream_len, lt_stream stream) {
+  lt_status st = check_shape(shape);
+  if (st != LT_OK) return st;
+  if (!mask || !aligned(K_stream, 16) || !aligned(V_stream, 16) || !aligned(stream_len, 4)) return LT_ERR_INVALID_ARG;
+  if (shape->total_tokens > 0 && (!aligned(K, 16) || !aligned(V, 16))) return LT_ERR_INVALID_ARG;
+  if (S < 0 || W < 0 || (long long)S + W < 1 || (long long)S + W > (1 << 24)) return LT_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != LT_OK) return st;
+  lt::CompactParams p;
+  p.batch = shape->batch;
+  p.total_tokens = shape->total_tokens;
+  p.hkv = shape->hkv;
+  p.D = shape->head_dim;
+  p.S = S;
+  p.W = W;
+  p.cu_seqlens = shape->cu_seqlens;
+  p.K = static_cast<const uint4*>(K);
+  p.V = static_cast<const uint4*>(V);
+  p.mask = mask;
+  p.Ks = static_cast<uint4*>(K_stream);
+  p.Vs = static_cast<uint4*>(V_stream);
+  p.len = stream_len;
+  const long long work = (long long)shape->batch * (S + W) * shape->hkv * (shape->head_dim / 8);
+  long long blocks = (work + 255) / 256;
+  const long long cap = (long long)dev->sm_count * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  lt::compact_kv_kernel<<<int(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_device_status(int clear) {
+  unsigned v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return LT_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof v) != cudaSuccess) return LT_ERR_CUDA;
+  if (clear) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero) != cudaSuccess) return LT_ERR_CUDA;
+  }
+  return (v & lt::kErrTimeout) ? LT_ERR_TIMEOUT : LT_OK;
+}
+
+}  // extern "C"

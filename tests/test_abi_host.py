@@ -1,0 +1,159 @@
+"""Host-side checks of the C ABI: the library loads, exports every function the
+header declares, rejects bad arguments before touching a device, and its host
+queue / selection agree with the oracle.  No GPU needed."""
+import ctypes
+import itertools
+import os
+import re
+
+import numpy as np
+import pytest
+
+import kv_cache_compression_tcgen05_b200 as lt
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    lt.build()
+    return lt.library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "lt.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lt_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert {"lt_prefill_attn", "lt_lazy_ratio", "lt_select_layers", "lt_compact_kv", "lt_queue_push"} <= set(names)
+    lib = ctypes.CDLL(lt.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_version():
+    assert lt.lt_status_string(lt.LT_OK) == "LT_OK"
+    assert lt.lt_status_string(lt.LT_ERR_TIMEOUT) == "LT_ERR_TIMEOUT"
+    assert lt.lt_version() >= 100
+
+
+def _shape(**kw):
+    s = lt.LtShape()
+    s.batch, s.total_tokens, s.max_seqlen, s.hq, s.hkv, s.head_dim = 1, 256, 256, 4, 2, 64
+    s.cu_seqlens = None
+    for k, v in kw.items():
+        setattr(s, k, v)
+    return s
+
+
+FAKE = 0x10000  # aligned, never dereferenced: every case below fails its checks first
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(head_dim=96), lt.LT_ERR_UNSUPPORTED),
+    (dict(head_dim=256), lt.LT_ERR_UNSUPPORTED),
+    (dict(hq=3, hkv=2), lt.LT_ERR_INVALID_ARG),
+    (dict(batch=0), lt.LT_ERR_INVALID_ARG),
+    (dict(batch=2), lt.LT_ERR_INVALID_ARG),       # batch > 1 needs cu_seqlens
+    (dict(total_tokens=-1), lt.LT_ERR_INVALID_ARG),
+    (dict(hkv=0), lt.LT_ERR_INVALID_ARG),
+])
+def test_prefill_attn_rejects_bad_shapes(kw, status):
+    s = _shape(**kw)
+    rc = lt.library().lt_prefill_attn(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, 0.0, None)
+    assert rc == status
+
+
+def test_calls_reject_null_and_misaligned_pointers():
+    lib = lt.library()
+    s = _shape()
+    assert lib.lt_prefill_attn(None, FAKE, FAKE, FAKE, FAKE, FAKE, 0.0, None) == lt.LT_ERR_INVALID_ARG
+    assert lib.lt_prefill_attn(ctypes.byref(s), None, FAKE, FAKE, FAKE, FAKE, 0.0, None) == lt.LT_ERR_INVALID_ARG
+    assert lib.lt_prefill_attn(ctypes.byref(s), FAKE + 8, FAKE, FAKE, FAKE, FAKE, 0.0, None) == lt.LT_ERR_INVALID_ARG
+    assert lib.lt_prefill_attn(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE + 2, 0.0, None) == lt.LT_ERR_INVALID_ARG
+    assert lib.lt_prefill_attn(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, float("nan"), None) == \
+        lt.LT_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("S,W,n_obs", [(0, 0, 16), (-1, 4, 16), (4, -2, 16), (4, 32, 0), (4, 32, 5000)])
+def test_lazy_ratio_rejects_bad_window(S, W, n_obs):
+    s = _shape()
+    rc = lt.library().lt_lazy_ratio(ctypes.byref(s), FAKE, FAKE, FAKE, 0.0, S, W, n_obs, FAKE, None)
+    assert rc == lt.LT_ERR_INVALID_ARG
+
+
+def test_lazy_ratio_rejects_huge_group():
+    s = _shape(hq=128, hkv=1)
+    assert lt.library().lt_lazy_ratio(ctypes.byref(s), FAKE, FAKE, FAKE, 0.0, 4, 32, 16, FAKE, None) == \
+        lt.LT_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("S,W", [(0, 0), (-1, 3), (2, -1)])
+def test_compact_rejects_bad_window(S, W):
+    s = _shape()
+    rc = lt.library().lt_compact_kv(ctypes.byref(s), FAKE, FAKE, FAKE, S, W, FAKE, FAKE, FAKE, None)
+    assert rc == lt.LT_ERR_INVALID_ARG
+
+
+def test_compact_rejects_null_mask():
+    s = _shape()
+    assert lt.library().lt_compact_kv(ctypes.byref(s), FAKE, FAKE, None, 4, 4, FAKE, FAKE, FAKE, None) == \
+        lt.LT_ERR_INVALID_ARG
+
+
+def test_layer_score_is_head_mean():
+    r = np.array([0.25, 0.5, 0.75, 1.0], np.float32)
+    assert abs(lt.lt_layer_score(r) - 0.625) < 1e-7
+
+
+def test_select_layers_matches_oracle():
+    rng = np.random.default_rng(3)
+    for L, B, H in ((4, 1, 2), (16, 3, 8), (64, 8, 40)):
+        ratios = rng.random((L, B, H)).astype(np.float32)
+        for budget in (0, 1, L // 2, L):
+            lazy, order = lt.lt_select_layers(ratios, budget)
+            scores = ratios.astype(np.float64).mean(axis=2).T    # float64 head means, as the C code sums
+            for b in range(B):
+                o_lazy, o_order = oracle.select_layers(np.array([lt.lt_layer_score(ratios[l, b]) for l in range(L)]),
+                                                       budget)
+                assert np.array_equal(lazy[b], o_lazy)
+                assert np.array_equal(order[b], o_order)
+                assert abs(scores[b] - [lt.lt_layer_score(ratios[l, b]) for l in range(L)]).max() < 1e-6
+
+
+def test_select_layers_rejects_nan_and_bad_budget():
+    r = np.ones((4, 1, 2), np.float32)
+    with pytest.raises(lt.LtError):
+        lt.lt_select_layers(r, 5)
+    r[2, 0, 1] = np.nan
+    with pytest.raises(lt.LtError):
+        lt.lt_select_layers(r, 2)
+
+
+def test_queue_matches_oracle_every_push_order():
+    rng = np.random.default_rng(5)
+    for L in range(1, 7):
+        scores = np.round(rng.random(L), 1).astype(np.float32)   # rounding makes ties likely
+        for budget in range(L + 1):
+            for perm in itertools.permutations(range(L)):
+                q = lt.LayerQueue(L, budget)
+                popped = [x for x in (q.push(l, scores[l]) for l in perm) if x >= 0]
+                want = oracle.queue_online(scores.astype(np.float64), budget, push_order=np.array(perm))
+                assert popped == want.tolist(), (scores, perm, budget)
+                assert len(q) == L - budget
+                q.close()
+
+
+def test_queue_rejects_bad_pushes():
+    q = lt.LayerQueue(4, 2)
+    assert q.push(0, 0.5) == -1
+    for layer, score in ((0, 0.1), (4, 0.1), (-1, 0.1), (1, float("nan")), (1, float("inf"))):
+        with pytest.raises(lt.LtError):
+            q.push(layer, score)
+    assert len(q) == 1
+    with pytest.raises(lt.LtError):
+        lt.lt_queue_create(3, 4)
