@@ -103,6 +103,23 @@ lt_status lt_prefill_attn(const lt_shape* shape, const void* Q, const void* K, c
                           float* LSE, float softmax_scale, lt_stream stream);
 
 /*
+ * The same attention fused with the lazy ratio: O and LSE as lt_prefill_attn,
+ * and ratio[b, h] as lt_lazy_ratio computes it (same S, W, n_obs and limits),
+ * accumulated inside the attention's online softmax: for the observed rows the
+ * weights of the keys in K_i are summed in the running-max frame of the
+ * softmax denominator, so r_i = num_i / l_i = sum_{j in K_i} exp(s_ij - LSE_i)
+ * with no second pass over the keys.  ratio: device fp32 [batch, hq], zeroed
+ * by this call on `stream` and then written.  For n_obs <= 128 the result is
+ * bitwise reproducible; above, the shares of more than two query tiles are
+ * added by atomics and may round differently from run to run.
+ * Sources: as lt_prefill_attn and lt_lazy_ratio (the write-up's first solution:
+ * the ratio rides on the prefill's own softmax statistics).
+ */
+lt_status lt_prefill_attn_ratio(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
+                                float* LSE, float softmax_scale, int S, int W, int n_obs, float* ratio,
+                                lt_stream stream);
+
+/*
  * Lazy ratio from the LSE.
  *   For every sequence b (length N), query head h and each of the last
  *   n' = min(n_obs, N) rows i of b:

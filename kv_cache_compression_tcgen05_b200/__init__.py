@@ -24,6 +24,7 @@ from .binding import (  # noqa: F401
     lt_layer_score,
     lt_lazy_ratio,
     lt_prefill_attn,
+    lt_prefill_attn_ratio,
     lt_queue_create,
     lt_queue_destroy,
     lt_queue_push,

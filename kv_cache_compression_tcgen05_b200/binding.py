@@ -46,6 +46,7 @@ _shp = ctypes.POINTER(LtShape)
 
 _SIGS = {
     "lt_prefill_attn": (_i, [_shp, _vp, _vp, _vp, _vp, _vp, _f, _vp]),
+    "lt_prefill_attn_ratio": (_i, [_shp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
     "lt_lazy_ratio": (_i, [_shp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
     "lt_layer_score": (_f, [_vp, _i]),
     "lt_select_layers": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
@@ -156,6 +157,37 @@ def lt_prefill_attn(Q, K, V, cu_seqlens=None, max_seqlen=None, softmax_scale=Non
                                      0.0 if softmax_scale is None else float(softmax_scale),
                                      _stream_handle(stream)), "lt_prefill_attn")
     return out, lse
+
+
+def lt_prefill_attn_ratio(Q, K, V, S, W, n_obs, cu_seqlens=None, max_seqlen=None, softmax_scale=None, out=None,
+                          lse=None, ratio=None, stream=None):
+    """Attention fused with the lazy ratio.  Returns (O [T, hq, d] bf16,
+    LSE [hq, T] fp32, ratio [batch, hq] fp32)."""
+    _dev_tensor(Q, "Q", torch.bfloat16, 3)
+    _dev_tensor(K, "K", torch.bfloat16, 3)
+    _dev_tensor(V, "V", torch.bfloat16, 3)
+    T, hq, d = Q.shape
+    hkv = K.shape[1]
+    if K.shape != (T, hkv, d) or V.shape != K.shape:
+        raise ValueError("K and V must be [T, hkv, d] with Q's T and d")
+    shape = _shape(T, hq, hkv, d, cu_seqlens, max_seqlen)
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty((hq, T), dtype=torch.float32, device=Q.device)
+    if ratio is None:
+        ratio = torch.empty((shape.batch, hq), dtype=torch.float32, device=Q.device)
+    _dev_tensor(out, "out", torch.bfloat16, 3)
+    _dev_tensor(lse, "lse", torch.float32, 2)
+    _dev_tensor(ratio, "ratio", torch.float32, 2)
+    if out.shape != Q.shape or lse.shape != (hq, T) or ratio.shape != (shape.batch, hq):
+        raise ValueError("out must be [T, hq, d], lse [hq, T] and ratio [batch, hq]")
+    _check(library().lt_prefill_attn_ratio(ctypes.byref(shape), Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                           out.data_ptr(), lse.data_ptr(),
+                                           0.0 if softmax_scale is None else float(softmax_scale), int(S), int(W),
+                                           int(n_obs), ratio.data_ptr(), _stream_handle(stream)),
+           "lt_prefill_attn_ratio")
+    return out, lse, ratio
 
 
 def lt_lazy_ratio(Q, K, LSE, S, W, n_obs, cu_seqlens=None, max_seqlen=None, softmax_scale=None, out=None,

@@ -1,28 +1,52 @@
-// attn_fwd.cuh -- causal GQA prefill attention with per-row LSE for sm_100a.
+// attn_fwd.cuh -- causal GQA prefill attention with per-row LSE (optionally
+// fused with the lazy ratio) for sm_100a.
 //
 // The LightTransfer write-up (xzbcqc.com news page, first solution of
 // LightTransfer-Test) reuses the log-sum-exp that a FlashAttention-style prefill
 // produces as the denominator of the lazy ratio.  This kernel is that prefill,
 // built for B200:
 //
-//   * persistent: one CTA per SM walks a list of (q-tile, sequence, head) work
-//     items, heaviest causal tiles first, in snake order across CTAs;
-//   * warp-specialised, 6 warps:
-//       warp 0      TMA producer: Q tile (double buffered) and a ring of K/V
-//                   tiles (128 keys x d, 128-byte swizzle), one mbarrier each;
-//       warp 1      owns the TMEM allocation; one thread issues tcgen05.mma:
-//                   S = Q K^T into one of two TMEM score buffers, then
-//                   O += P V into the TMEM output accumulator;
-//       warps 2..5  softmax: thread = query row = TMEM lane.  tcgen05.ld of the
-//                   128 scores, causal mask on the diagonal tile, running max
-//                   in the log2 domain, exp2, bf16 P written to shared memory in
-//                   the MMA's swizzled K-major layout, lazy O rescale (only when
-//                   the running max grows by more than 2^8), epilogue O / l and
-//                   LSE = (m + log2 l) ln 2 written once.
-//   * tiles: 128 query rows x 128 keys; M = 128, N = 128 (S) and N = d (PV),
-//     K-step 16 per tcgen05.mma.
+//   * persistent: one CTA per SM walks a list of work items, heaviest first,
+//     snake-ordered across CTAs.  A work item is two 128-row query tiles that
+//     read the same K/V stream: two query heads of one KV head at the same
+//     q-tile when the GQA group is even, otherwise two consecutive q-tiles of
+//     one head (the earlier tile then skips the last key tile).
+//   * warp-specialised, 10 warps:
+//       warp 0      TMA producer: the item's two Q tiles (double buffered) and
+//                   a ring of K/V tiles (128 keys x d, 128-byte swizzle);
+//       warp 1      owns the TMEM allocation; one thread issues every tcgen05.mma
+//                   in the order  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), ...
+//                   so the tensor core works for one tile while the other
+//                   tile's softmax runs;
+//       warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: thread =
+//                   query row = TMEM lane.  tcgen05.ld of the 128 scores, causal
+//                   mask on the diagonal tile, running max in the log2 domain
+//                   (the O accumulator is rescaled only when the max grows by
+//                   more than 2^8; exact, because O and l share the stale max),
+//                   exp2, bf16 P written back over the scores in TMEM with
+//                   tcgen05.st (P is the A operand of O += P V, read from TMEM);
+//                   epilogue O / l and LSE = (m + log2 l) ln 2, written once.
+//   * d = 128, TMEM [0,128) S/P of A, [128,256) S/P of B, [256,384) O of A,
+//     [384,512) O of B.  P overwrites the first half of its S columns; the MMAs
+//     of one thread execute in issue order, so S_X(j+1), issued after PV_X(j),
+//     never overwrites P_X(j) before PV_X(j) has read it, and once S_X(j+1) is
+//     complete so is PV_X(j): the softmax may rescale O_X right away.
+//   * d = 64, TMEM S [0,128) [128,256), P [256,320) [320,384), O [384,448)
+//     [448,512).  With P in its own columns the softmax frees S as soon as the
+//     scores are in registers, and S_X(j+1) runs on the tensor core while the
+//     softmax of tile j is still exponentiating; the softmax waits for PV_X(j-1)
+//     only before it overwrites P and rescales O.
 //
-// TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256, 256+d) O.
+// Fused lazy ratio (press-release page, "LightTransfer方法详解": attention
+// weights from the query to the initial and the recent keys): for the last
+// n_obs rows of each sequence the softmax threads also sum, in the same
+// stale-max frame as l, the weights of the keys
+//     K_i = [0, min(S, i+1)) U [max(S, i-W+1), i],
+// so r_i = num_i / l_i = sum_{j in K_i} exp(s_ij - LSE_i).  The rows of a tile
+// are added in a fixed order (lanes, then the tile's four warps) and one
+// atomic add per (tile, head) puts the tile's share of the mean into
+// ratio[b, h]; with n_obs <= 128 at most two tiles touch a (b, h), and a
+// two-term sum does not depend on the order.
 #pragma once
 
 #include "lt_device.cuh"
@@ -34,95 +58,153 @@ struct AttnParams {
   int total_tokens;
   int hq;
   int hkv;
+  int group;        // hq / hkv
   int n_qtiles;     // ceil(max_seqlen / 128)
-  int num_tiles;    // n_qtiles * batch * hq
+  int pair_heads;   // 1: an item pairs two heads; 0: it pairs two q-tiles
+  int num_items;
   const int32_t* cu_seqlens;  // device [batch+1] or null (one sequence)
   __nv_bfloat16* O;
   float* LSE;
   float scale_log2;  // softmax scale * log2(e)
   unsigned* status;
+  // fused lazy ratio
+  float* ratio;      // [batch, hq], zeroed before the launch
+  int S;
+  int W;
+  int n_obs;
 };
 
 template <int D>
 struct AttnLayout {
-  static constexpr int kBlock = 128;                  // query rows = keys per tile
-  static constexpr int kTileBytes = kBlock * D * 2;   // one Q, K or V tile
+  static constexpr int kTileBytes = 128 * D * 2;      // one Q, K or V tile
   static constexpr int kSub = 16384;                  // one 128 x 64 bf16 swizzled sub-tile
-  static constexpr int kStages = D == 64 ? 4 : 3;     // K/V ring slots
-  static constexpr int kPBytes = kBlock * kBlock * 2;
-  static constexpr int kQOff = 0;
-  static constexpr int kRingOff = kQOff + 2 * kTileBytes;
-  static constexpr int kPOff = kRingOff + kStages * kTileBytes;
-  static constexpr int kBarOff = kPOff + 2 * kPBytes;
-  static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 1 + 1;
+  static constexpr int kStages = D == 64 ? 6 : 3;     // K/V ring slots
+  static constexpr int kQOff = 0;                     // [2 buffers][2 tiles]
+  static constexpr int kRingOff = kQOff + 4 * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
+  static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 2 + 2 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kBytes = kMiscOff + 64;
   static constexpr int kAlloc = kBytes + 1024;        // room to align the base to 1024 B
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kTmemO = 256;
+  // d = 64: P of each tile has its own 64 columns, so S(j+1) may be written while
+  // P(j) waits for its MMA: S [0,128) [128,256), P [256,320) [320,384),
+  // O [384,448) [448,512).  d = 128: P overwrites the first half of its S
+  // columns: S/P [0,128) [128,256), O [256,384) [384,512).
+  static constexpr bool kSepP = D == 64;
+  static constexpr uint32_t kTmemP = kSepP ? 256 : 0;
+  static constexpr uint32_t kPStride = kSepP ? 64 : 128;
+  static constexpr uint32_t kTmemO = kSepP ? 384 : 256;
 };
 
-struct AttnTile {
-  int b, h, qt, start, len;
+struct AttnItem {
+  int b, kh, start, len;
+  int h[2], qt[2], n[2];
+  bool hasB;
 };
 
-// Work item t -> (sequence, head, q-tile); false when the q-tile lies beyond the
-// sequence.  Items are ordered heaviest q-tile first; within one q-tile the
-// heads of one sequence are consecutive, so CTAs running at the same time share
-// K/V tiles through L2.
-__device__ __forceinline__ bool attn_decode(const AttnParams& p, int t, AttnTile& tile) {
-  const int bh = p.batch * p.hq;
-  tile.qt = p.n_qtiles - 1 - t / bh;
-  const int rem = t - (t / bh) * bh;
-  tile.b = rem / p.hq;
-  tile.h = rem - tile.b * p.hq;
+__device__ __forceinline__ void seq_bounds(const AttnParams& p, int b, int& start, int& len) {
   if (p.cu_seqlens) {
-    tile.start = p.cu_seqlens[tile.b];
-    tile.len = p.cu_seqlens[tile.b + 1] - tile.start;
+    start = p.cu_seqlens[b];
+    len = p.cu_seqlens[b + 1] - start;
   } else {
-    tile.start = 0;
-    tile.len = p.total_tokens;
+    start = 0;
+    len = p.total_tokens;
   }
-  return tile.qt * 128 < tile.len;
+}
+
+// Work item t -> its one or two tiles; false when the item has no valid tile.
+// Items are ordered heaviest first; the items of one q position are consecutive
+// (heads of a sequence next to each other, so concurrent CTAs share K/V in L2).
+__device__ __forceinline__ bool attn_decode(const AttnParams& p, int t, AttnItem& it) {
+  if (p.pair_heads) {
+    const int hp_count = p.hq >> 1;
+    const int per_q = p.batch * hp_count;
+    const int qt = p.n_qtiles - 1 - t / per_q;
+    const int rem = t - (t / per_q) * per_q;
+    it.b = rem / hp_count;
+    const int hp = rem - it.b * hp_count;
+    seq_bounds(p, it.b, it.start, it.len);
+    it.h[0] = 2 * hp;
+    it.h[1] = 2 * hp + 1;
+    it.qt[0] = it.qt[1] = qt;
+    it.n[0] = it.n[1] = qt + 1;
+    it.hasB = true;
+    it.kh = it.h[0] / p.group;
+    return qt * 128 < it.len;
+  }
+  const int per_q = p.batch * p.hq;
+  const int npairs = (p.n_qtiles + 1) >> 1;
+  const int qp = npairs - 1 - t / per_q;
+  const int rem = t - (t / per_q) * per_q;
+  it.b = rem / p.hq;
+  const int h = rem - it.b * p.hq;
+  seq_bounds(p, it.b, it.start, it.len);
+  it.h[0] = it.h[1] = h;
+  it.kh = h / p.group;
+  const int t1 = 2 * qp + 1, t0 = 2 * qp;
+  if (t1 * 128 < it.len) {
+    it.qt[0] = t1;
+    it.qt[1] = t0;
+    it.n[0] = t1 + 1;
+    it.n[1] = t0 + 1;
+    it.hasB = true;
+    return true;
+  }
+  it.qt[0] = it.qt[1] = t0;
+  it.n[0] = it.n[1] = t0 + 1;
+  it.hasB = false;
+  return t0 * 128 < it.len;
 }
 
 // Snake order: CTA c takes item k*G + c on even rounds and k*G + (G-1-c) on odd
 // rounds, so the heaviest items are spread evenly.
-__device__ __forceinline__ int attn_item(int round, int cta, int grid) {
+__device__ __forceinline__ int attn_item_index(int round, int cta, int grid) {
   return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
 }
 
-template <int D>
+// Every kEmuPeriod-th pair of softmax columns takes the FMA-pipe exp2 (0: none).
+constexpr int kEmuPeriod = 0;
+
+template <bool V>
+struct BoolConst {
+  static constexpr bool value = V;
+};
+
+template <int D, bool kRatio>
 __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using Lay = AttnLayout<D>;
+  constexpr bool kSepP = Lay::kSepP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + Lay::kQOff;
   uint8_t* sRing = smem + Lay::kRingOff;
-  uint8_t* sP = smem + Lay::kPOff;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBarOff);
-  uint64_t* q_full = bars;                       // [2]  TMA -> MMA
-  uint64_t* q_empty = q_full + 2;                // [2]  MMA -> TMA
+  uint64_t* q_full = bars;                       // [2 buffers]   TMA -> MMA
+  uint64_t* q_empty = q_full + 2;                // [2 buffers]   MMA -> TMA
   uint64_t* kv_full = q_empty + 2;               // [kStages]
   uint64_t* kv_empty = kv_full + Lay::kStages;   // [kStages]
-  uint64_t* s_full = kv_empty + Lay::kStages;    // [2]  MMA -> softmax
-  uint64_t* p_full = s_full + 2;                 // [2]  softmax -> MMA (128 arrivals)
-  uint64_t* pv_done = p_full + 2;                // [2]  MMA -> softmax
-  uint64_t* o_empty = pv_done + 2;               // [1]  softmax -> MMA (128 arrivals)
-  uint64_t* drain = o_empty + 1;                 // [1]  MMA drain on abort
+  uint64_t* s_full = kv_empty + Lay::kStages;    // [2 tiles]     MMA -> softmax
+  uint64_t* p_full = s_full + 2;                 // [2 tiles]     softmax -> MMA (128 arrivals)
+  uint64_t* o_full = p_full + 2;                 // [2 tiles]     MMA -> epilogue
+  uint64_t* o_empty = o_full + 2;                // [2 tiles]     epilogue -> MMA (128 arrivals)
+  uint64_t* s_free = o_empty + 2;                // [2 tiles]     softmax -> MMA (128 arrivals; d = 64)
+  uint64_t* pv_done = s_free + 2;                // [2 tiles]     MMA -> softmax (d = 64)
+  uint64_t* drain = pv_done + 2;                 // [1]           MMA drain on abort
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
   // Never raised: the drain waits after an abort end on completion or time only.
   volatile int* no_abort = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 8);
+  float* ratio_part = reinterpret_cast<float*>(smem + Lay::kMiscOff + 16);   // [2 tiles][4 warps]
+  int* ratio_cnt = reinterpret_cast<int*>(smem + Lay::kMiscOff + 48);        // [2 tiles] warps done
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int grid = gridDim.x;
   const int cta = blockIdx.x;
-  const int group = p.hq / p.hkv;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -130,16 +212,19 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 128);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], 128);
+      mbar_init(&s_free[i], 128);
       mbar_init(&pv_done[i], 1);
     }
     for (int i = 0; i < Lay::kStages; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(o_empty, 128);
     mbar_init(drain, 1);
     *abort_flag = 0;
     *no_abort = 0;
+    ratio_cnt[0] = ratio_cnt[1] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -154,50 +239,45 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl ctl{abort_flag, p.status};
-
+  const WaitCtl drain_ctl{no_abort, p.status};
   if (warp == 0) {
     // ------------------------------------------------------------- producer
     if (lane == 0) {
-      int it = 0, tl = 0;
+      int ring = 0, nq = 0;
       bool ok = true;
-      for (int round = 0; ok && round * grid < p.num_tiles; ++round) {
-        const int t = attn_item(round, cta, grid);
-        AttnTile tile;
-        if (t >= p.num_tiles || !attn_decode(p, t, tile)) continue;
-        const int qb = tl & 1;
-        if (tl >= 2 && !(ok = mbar_wait(&q_empty[qb], ((tl >> 1) - 1) & 1, ctl))) break;
-        mbar_expect_tx(&q_full[qb], Lay::kTileBytes);
-        for (int st = 0; st < D / 64; ++st)
-          tma_load_3d(sQ + qb * Lay::kTileBytes + st * Lay::kSub, &tmQ, &q_full[qb], st * 64, tile.h,
-                      tile.start + tile.qt * 128);
-        const int n = tile.qt + 1;
-        const int kh = tile.h / group;
-        // Order of use by the MMA thread: K0, K1, V0, K2, V1, ..., V(n-1).
-        for (int step = 0; ok && step <= n; ++step) {
-          for (int which = 0; which < 2; ++which) {
-            const bool isK = which == 0;
-            if (isK ? step >= n : step < 1) continue;
-            const int j = isK ? step : step - 1;
-            const int slot = it % Lay::kStages;
-            if (it >= Lay::kStages && !(ok = mbar_wait(&kv_empty[slot], ((it / Lay::kStages) - 1) & 1, ctl)))
+      for (int round = 0; ok && round * grid < p.num_items; ++round) {
+        const int t = attn_item_index(round, cta, grid);
+        AttnItem it;
+        if (t >= p.num_items || !attn_decode(p, t, it)) continue;
+        const int qb = nq & 1;
+        if (nq >= 2 && !(ok = mbar_wait(&q_empty[qb], ((nq >> 1) - 1) & 1, ctl))) break;
+        const int ntile = it.hasB ? 2 : 1;
+        mbar_expect_tx(&q_full[qb], ntile * Lay::kTileBytes);
+        for (int x = 0; x < ntile; ++x)
+          for (int st = 0; st < D / 64; ++st)
+            tma_load_3d(sQ + (qb * 2 + x) * Lay::kTileBytes + st * Lay::kSub, &tmQ, &q_full[qb], st * 64, it.h[x],
+                        it.start + it.qt[x] * 128);
+        ++nq;
+        // Ring order: K0, V0, K1, V1, ...
+        for (int j = 0; ok && j < it.n[0]; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const int slot = ring % Lay::kStages;
+            if (ring >= Lay::kStages && !(ok = mbar_wait(&kv_empty[slot], ((ring / Lay::kStages) - 1) & 1, ctl)))
               break;
             mbar_expect_tx(&kv_full[slot], Lay::kTileBytes);
             for (int st = 0; st < D / 64; ++st)
-              tma_load_3d(sRing + slot * Lay::kTileBytes + st * Lay::kSub, isK ? &tmK : &tmV, &kv_full[slot],
-                          st * 64, kh, tile.start + j * 128);
-            ++it;
+              tma_load_3d(sRing + slot * Lay::kTileBytes + st * Lay::kSub, kv == 0 ? &tmK : &tmV, &kv_full[slot],
+                          st * 64, it.kh, it.start + j * 128);
+            ++ring;
           }
         }
-        ++tl;
       }
       if (!ok) {
         // Let the loads already issued land before the CTA's shared memory is
         // released (bounded; the abort flag is ignored here).
-        const int first = it > Lay::kStages ? it - Lay::kStages : 0;
-        for (int x = first; x < it; ++x) {
-          const WaitCtl drain_ctl{no_abort, p.status};
+        for (int x = ring > Lay::kStages ? ring - Lay::kStages : 0; x < ring; ++x)
           mbar_wait(&kv_full[x % Lay::kStages], (x / Lay::kStages) & 1, drain_ctl);
-        }
+        for (int x = nq > 2 ? nq - 2 : 0; x < nq; ++x) mbar_wait(&q_full[x & 1], (x >> 1) & 1, drain_ctl);
       }
     }
   } else if (warp == 1) {
@@ -205,119 +285,169 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
-      int it = 0, js = 0, tl = 0;
+      int ring = 0, nq = 0;
+      int cnt_p0 = 0, cnt_p1 = 0;   // P tiles consumed, per tile slot
+      int cnt_s0 = 0, cnt_s1 = 0;   // S tiles issued, per tile slot (d = 64)
+      int cnt_o0 = 0, cnt_o1 = 0;   // items finished, per tile slot
       bool ok = true;
-      for (int round = 0; ok && round * grid < p.num_tiles; ++round) {
-        const int t = attn_item(round, cta, grid);
-        AttnTile tile;
-        if (t >= p.num_tiles || !attn_decode(p, t, tile)) continue;
-        const int qb = tl & 1;
-        if (!(ok = mbar_wait(&q_full[qb], (tl >> 1) & 1, ctl))) break;
-        const uint32_t q_addr = smem_u32(sQ + qb * Lay::kTileBytes);
-        const int n = tile.qt + 1;
-
-        auto issue_s = [&](int g) -> bool {
-          const int slot = it % Lay::kStages;
-          if (!mbar_wait(&kv_full[slot], (it / Lay::kStages) & 1, ctl)) return false;
+      for (int round = 0; ok && round * grid < p.num_items; ++round) {
+        const int t = attn_item_index(round, cta, grid);
+        AttnItem it;
+        if (t >= p.num_items || !attn_decode(p, t, it)) continue;
+        const int qb = nq & 1;
+        if (!(ok = mbar_wait(&q_full[qb], (nq >> 1) & 1, ctl))) break;
+        ++nq;
+        const int base = ring;
+        const int n = it.n[0];
+        const int nB = it.hasB ? it.n[1] : 0;
+        auto slot_of = [&](int j, int kv) { return (base + 2 * j + kv) % Lay::kStages; };
+        auto phase_of = [&](int j, int kv) { return ((base + 2 * j + kv) / Lay::kStages) & 1; };
+        // S_x(j) = Q_x K_j^T into the tile's TMEM score columns.
+        auto issue_s = [&](int x, int j) -> bool {
+          const int slot = slot_of(j, 0);
+          if constexpr (kSepP) {
+            // The softmax must have loaded the previous scores of this tile.
+            int& cnt_s = x ? cnt_s1 : cnt_s0;
+            if (cnt_s > 0 && !mbar_wait(&s_free[x], (cnt_s - 1) & 1, ctl)) return false;
+            ++cnt_s;
+          }
+          if (x == 0) {   // tile A always uses K_j first
+            if (!mbar_wait(&kv_full[slot], phase_of(j, 0), ctl)) return false;
+          }
           tc_fence_after();
+          const uint32_t q_addr = smem_u32(sQ + (qb * 2 + x) * Lay::kTileBytes);
           const uint32_t k_addr = smem_u32(sRing + slot * Lay::kTileBytes);
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t off = (k >> 2) * Lay::kSub + (k & 3) * 32;
-            mma_bf16_ss(tmem + (g & 1) * 128, smem_desc_sw128(q_addr + off, 16, 1024),
+            mma_bf16_ss(tmem + x * 128, smem_desc_sw128(q_addr + off, 16, 1024),
                         smem_desc_sw128(k_addr + off, 16, 1024), kIdS, k > 0 ? 1u : 0u);
           }
-          mma_commit(&kv_empty[slot]);
-          mma_commit(&s_full[g & 1]);
-          ++it;
+          mma_commit(&s_full[x]);
+          const bool last_use = x == 1 || j >= nB;
+          if (last_use) mma_commit(&kv_empty[slot]);
+          if (last_use && j == n - 1) mma_commit(&q_empty[qb]);
           return true;
         };
-        auto issue_pv = [&](int g, int j) -> bool {
-          if (!mbar_wait(&p_full[g & 1], (g >> 1) & 1, ctl)) return false;
-          if (j == 0 && tl > 0 && !mbar_wait(o_empty, (tl - 1) & 1, ctl)) return false;
-          const int slot = it % Lay::kStages;
-          if (!mbar_wait(&kv_full[slot], (it / Lay::kStages) & 1, ctl)) return false;
+        // O_x += P_x(j) V_j, P_x(j) read from TMEM.
+        auto issue_pv = [&](int x, int j) -> bool {
+          int& cnt_p = x ? cnt_p1 : cnt_p0;
+          int& cnt_o = x ? cnt_o1 : cnt_o0;
+          if (!mbar_wait(&p_full[x], cnt_p & 1, ctl)) return false;
+          ++cnt_p;
+          if (j == 0 && cnt_o > 0 && !mbar_wait(&o_empty[x], (cnt_o - 1) & 1, ctl)) return false;
+          const int slot = slot_of(j, 1);
+          if (x == 0 && !mbar_wait(&kv_full[slot], phase_of(j, 1), ctl)) return false;
           tc_fence_after();
-          const uint32_t p_addr = smem_u32(sP + (g & 1) * Lay::kPBytes);
           const uint32_t v_addr = smem_u32(sRing + slot * Lay::kTileBytes);
 #pragma unroll
           for (int k = 0; k < 128 / 16; ++k) {
-            const uint64_t a = smem_desc_sw128(p_addr + (k >> 2) * Lay::kSub + (k & 3) * 32, 16, 1024);
             const uint64_t b = smem_desc_sw128(v_addr + k * 2048, Lay::kSub, 1024);
-            mma_bf16_ss(tmem + Lay::kTmemO, a, b, kIdPV, (j > 0 || k > 0) ? 1u : 0u);
+            mma_bf16_ts(tmem + Lay::kTmemO + x * D, tmem + Lay::kTmemP + x * Lay::kPStride + k * 8, b, kIdPV,
+                        (j > 0 || k > 0) ? 1u : 0u);
           }
-          mma_commit(&kv_empty[slot]);
-          mma_commit(&pv_done[g & 1]);
-          ++it;
+          if constexpr (kSepP) mma_commit(&pv_done[x]);
+          const bool last_use = x == 1 || j >= nB;
+          if (last_use) mma_commit(&kv_empty[slot]);
+          if ((x == 0 && j == n - 1) || (x == 1 && j == nB - 1)) {
+            mma_commit(&o_full[x]);
+            ++cnt_o;
+          }
           return true;
         };
 
-        if (!(ok = issue_s(js))) break;
-        if (n == 1) mma_commit(&q_empty[qb]);
-        for (int j = 0; ok && j < n; ++j) {
-          if (j + 1 < n) {
-            if (!(ok = issue_s(js + j + 1))) break;
-            if (j + 2 == n) mma_commit(&q_empty[qb]);
+        ok = issue_s(0, 0) && (nB == 0 || issue_s(1, 0));
+        if constexpr (kSepP) {
+          // S(j+1) as soon as the softmax has read S(j); PV(j) once P(j) is written.
+          for (int j = 0; ok && j < n; ++j) {
+            if (j + 1 < n) ok = issue_s(0, j + 1);
+            if (ok && j + 1 < nB) ok = issue_s(1, j + 1);
+            if (ok) ok = issue_pv(0, j);
+            if (ok && j < nB) ok = issue_pv(1, j);
           }
-          ok = issue_pv(js + j, j);
+        } else {
+          // P(j) overwrites S(j): PV(j) must be issued before S(j+1).
+          for (int j = 0; ok && j < n; ++j) {
+            ok = issue_pv(0, j) && (j + 1 >= n || issue_s(0, j + 1));
+            if (ok && j < nB) ok = issue_pv(1, j) && (j + 1 >= nB || issue_s(1, j + 1));
+          }
         }
-        js += n;
-        ++tl;
+        ring = base + 2 * n;
       }
       if (!ok) {
         mma_commit(drain);
-        const WaitCtl drain_ctl{no_abort, p.status};
         mbar_wait(drain, 0, drain_ctl);
       }
     }
   } else {
     // --------------------------------------------------------------- softmax
-    const int wq = warp & 3;                  // TMEM lane quarter of this warp
-    const int row = wq * 32 + lane;           // query row within the tile
+    const int x = (warp - 2) >> 2;             // tile slot: 0 = A (warps 2..5), 1 = B (warps 6..9)
+    const int wq = warp & 3;                   // TMEM lane quarter of this warp
+    const int row = wq * 32 + lane;            // query row within the tile
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
+    const uint32_t s_col = tmem + lane_off + x * 128;
+    const uint32_t p_col = tmem + lane_off + Lay::kTmemP + x * Lay::kPStride;
+    const uint32_t o_col = tmem + lane_off + Lay::kTmemO + x * D;
     const float sl2 = p.scale_log2;
-    int js = 0, tl = 0;
+    int cnt_s = 0, cnt_o = 0;
     bool ok = true;
-    for (int round = 0; ok && round * grid < p.num_tiles; ++round) {
-      const int t = attn_item(round, cta, grid);
-      AttnTile tile;
-      if (t >= p.num_tiles || !attn_decode(p, t, tile)) continue;
-      const int n = tile.qt + 1;
-      const int qpos = tile.qt * 128 + row;
+    for (int round = 0; ok && round * grid < p.num_items; ++round) {
+      const int t = attn_item_index(round, cta, grid);
+      AttnItem it;
+      if (t >= p.num_items || !attn_decode(p, t, it)) continue;
+      if (x == 1 && !it.hasB) continue;
+      const int qt = x ? it.qt[1] : it.qt[0];   // selects, not a local-memory index
+      const int n = x ? it.n[1] : it.n[0];
+      const int h = x ? it.h[1] : it.h[0];
+      const int qpos = qt * 128 + row;
+      // Fused ratio: is this row one of the last n_obs rows of its sequence?
+      int n_obs_seq = 0, obs_lo = 0;
+      bool tile_obs = false, row_obs = false;
+      if constexpr (kRatio) {
+        n_obs_seq = min(p.n_obs, it.len);
+        obs_lo = it.len - n_obs_seq;
+        tile_obs = qt * 128 + 127 >= obs_lo && qt * 128 < it.len;
+        row_obs = tile_obs && qpos >= obs_lo && qpos < it.len;
+      }
       float m_run = -INFINITY;   // running max of scale*log2(e)*s, possibly stale by < 8
       float l_run = 0.f;         // running sum of exp2(.. - m_run)
+      float num = 0.f;           // fused ratio numerator, same frame as l_run
       for (int j = 0; j < n; ++j) {
-        const int g = js + j;
-        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[g & 1], (g >> 1) & 1, ctl));
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x], cnt_s & 1, ctl));
         if (!ok) break;
+        ++cnt_s;
         tc_fence_after();
+        const bool diag = j == qt;
+        // All 128 scores of the row in one batch of TMEM loads (a single
+        // wait: the load latency is paid once per tile).
         uint32_t sr[128];
         {
           uint32_t(&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
           uint32_t(&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
           uint32_t(&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
           uint32_t(&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
-          const uint32_t sa = tmem + lane_off + (g & 1) * 128;
-          tmem_ld32(sa + 0, c0);
-          tmem_ld32(sa + 32, c1);
-          tmem_ld32(sa + 64, c2);
-          tmem_ld32(sa + 96, c3);
+          tmem_ld32(s_col + 0, c0);
+          tmem_ld32(s_col + 32, c1);
+          tmem_ld32(s_col + 64, c2);
+          tmem_ld32(s_col + 96, c3);
           tmem_wait_ld();
         }
-        float s[128];
-#pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-        if (j == tile.qt) {
+        if constexpr (kSepP) {
+          // The scores are in registers: the MMA may overwrite S with S(j+1).
+          tc_fence_before();
+          mbar_arrive(&s_free[x]);
+        }
+        if (diag) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (c > row) s[c] = -INFINITY;
+            if (c > row) sr[c] = __float_as_uint(-INFINITY);
         }
-        // Row maximum as 8 independent chains (short dependency chains).
+        // Row maximum as 8 independent chains.
         float mx8[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+        for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(sr[k]);
 #pragma unroll
-        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_new = fmaxf(m_run, mx * sl2);
@@ -328,64 +458,93 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
           m_run = m_new;
         }
         l_run *= alpha;
-        uint32_t pk[64];
-        float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const float neg_m = -m_run;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float p0 = fast_exp2(fmaf(s[2 * c], sl2, neg_m));
-          const float p1 = fast_exp2(fmaf(s[2 * c + 1], sl2, neg_m));
-          sum8[c & 7] += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
-        }
-        l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-        // The P buffer of this tile was last read by PV(g-2).
-        if (g >= 2) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[g & 1], ((g - 2) >> 1) & 1, ctl));
-          if (!ok) break;
-        }
-        {
-          const uint32_t pbase = smem_u32(sP + (g & 1) * Lay::kPBytes) + row * 128;
-#pragma unroll
-          for (int ch = 0; ch < 16; ++ch) {
-            const uint32_t addr = pbase + (ch >> 3) * Lay::kSub + (uint32_t(((ch & 7) ^ (row & 7))) << 4);
-            st_shared_v4(addr, pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+        if constexpr (kRatio) num *= alpha;
+        if constexpr (kSepP) {
+          // P(j) reuses the P columns and O(j) accumulates onto O: both need PV(j-1) done.
+          if (cnt_s > 1) {   // cnt_s - 1 = index of this tile among the slot's tiles
+            ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (cnt_s - 2) & 1, ctl));
+            if (!ok) break;
+            tc_fence_after();
           }
         }
-        fence_proxy_async_smem();
+        // exp2 in 32-column chunks; each chunk's bf16 P goes to TMEM (16
+        // columns) as soon as it is packed.  Every kEmuPeriod-th pair of
+        // columns may use the FMA-pipe exp2 to share work with the MUFU unit.
+        float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float neg_m = -m_run;
+        float racc = 0.f;
+        bool band = false;
+        int win_lo = 0;
+        if constexpr (kRatio) {
+          win_lo = qpos - p.W + 1;
+          band = row_obs && (j * 128 < p.S || j * 128 + 127 >= win_lo);
+        }
+        auto exp_chunks = [&](auto with_band) {
+          constexpr bool kBand = decltype(with_band)::value;
+#pragma unroll
+          for (int cb = 0; cb < 4; ++cb) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int c0 = cb * 32 + 2 * c;
+              const float x0 = fmaf(__uint_as_float(sr[c0]), sl2, neg_m);
+              const float x1 = fmaf(__uint_as_float(sr[c0 + 1]), sl2, neg_m);
+              float p0, p1;
+              if (kEmuPeriod > 0 && (c % kEmuPeriod) == kEmuPeriod - 1) {
+                p0 = exp2_fma(x0);
+                p1 = exp2_fma(x1);
+              } else {
+                p0 = fast_exp2(x0);
+                p1 = fast_exp2(x1);
+              }
+              sum8[c & 7] += p0 + p1;
+              pk[c] = pack_bf16x2(p0, p1);
+              if constexpr (kBand) {
+                // Weights of the sink keys and the W most recent keys of this row.
+                const int k0 = j * 128 + c0, k1 = k0 + 1;
+                racc += (k0 <= qpos && (k0 < p.S || k0 >= win_lo)) ? p0 : 0.f;
+                racc += (k1 <= qpos && (k1 < p.S || k1 >= win_lo)) ? p1 : 0.f;
+              }
+            }
+            tmem_st16(p_col + cb * 16, pk);
+          }
+        };
+        if (kRatio && __any_sync(0xffffffffu, band))
+          exp_chunks(BoolConst<true>{});
+        else
+          exp_chunks(BoolConst<false>{});
+        l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+        if constexpr (kRatio) num += band ? racc : 0.f;
         if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // Rescale the output accumulator once PV(g-1) has landed in it.
-          ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, ctl));
-          if (!ok) break;
-          tc_fence_after();
+          // PV(j-1) is complete (d = 128: S(j) was issued after it; d = 64: waited
+          // on above): rescale O in TMEM before PV(j) accumulates onto it.
 #pragma unroll
           for (int cb = 0; cb < D / 32; ++cb) {
             uint32_t o[32];
-            const uint32_t oa = tmem + lane_off + Lay::kTmemO + cb * 32;
-            tmem_ld32(oa, o);
+            tmem_ld32(o_col + cb * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(oa, o);
+            tmem_st32(o_col + cb * 32, o);
           }
-          tmem_wait_st();
         }
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&p_full[g & 1]);
+        mbar_arrive(&p_full[x]);
       }
       if (!ok) break;
       // --------------------------------------------------------- epilogue
-      const int gl = js + n - 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[gl & 1], (gl >> 1) & 1, ctl));
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_full[x], cnt_o & 1, ctl));
       if (!ok) break;
+      ++cnt_o;
       tc_fence_after();
-      const bool valid = qpos < tile.len;
+      const bool valid = qpos < it.len;
       const float inv_l = 1.f / l_run;
-      const size_t orow = (size_t(tile.start) + qpos) * p.hq + tile.h;
+      const size_t orow = (size_t(it.start) + qpos) * p.hq + h;
 #pragma unroll
       for (int cb = 0; cb < D / 32; ++cb) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_off + Lay::kTmemO + cb * 32, o);
+        tmem_ld32(o_col + cb * 32, o);
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
@@ -398,11 +557,30 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
         }
       }
       if (valid)
-        p.LSE[size_t(tile.h) * p.total_tokens + tile.start + qpos] = (m_run + fast_log2(l_run)) * 0.69314718055994531f;
+        p.LSE[size_t(h) * p.total_tokens + it.start + qpos] = (m_run + fast_log2(l_run)) * 0.69314718055994531f;
       tc_fence_before();
-      mbar_arrive(o_empty);
-      js += n;
-      ++tl;
+      mbar_arrive(&o_empty[x]);
+      if constexpr (kRatio) {
+        if (tile_obs) {
+          // This tile's share of mean_i r_i: its rows added in a fixed order.
+          float r = row_obs ? num * inv_l : 0.f;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+          // No barrier (a sibling warp may have left on a timed-out wait): the
+          // fourth warp to finish adds the four partials in warp order.
+          if (lane == 0) {
+            ratio_part[x * 4 + wq] = r;
+            __threadfence_block();
+            if (atomicAdd(&ratio_cnt[x], 1) == 3) {
+              __threadfence_block();
+              const volatile float* part = ratio_part + x * 4;
+              const float tot = (part[0] + part[1]) + (part[2] + part[3]);
+              atomicAdd(p.ratio + size_t(it.b) * p.hq + h, tot / float(n_obs_seq));
+              ratio_cnt[x] = 0;
+            }
+          }
+        }
+      }
     }
   }
 

@@ -46,9 +46,13 @@ lt_status device_info(DeviceInfo** out) {
     void* addr = nullptr;
     if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess) return LT_ERR_CUDA;
     info.status = static_cast<unsigned*>(addr);
-    if (cudaFuncSetAttribute(lt::attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(lt::attn_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              lt::AttnLayout<64>::kAlloc) != cudaSuccess ||
-        cudaFuncSetAttribute(lt::attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(lt::attn_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             lt::AttnLayout<128>::kAlloc) != cudaSuccess ||
+        cudaFuncSetAttribute(lt::attn_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             lt::AttnLayout<64>::kAlloc) != cudaSuccess ||
+        cudaFuncSetAttribute(lt::attn_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              lt::AttnLayout<128>::kAlloc) != cudaSuccess ||
         cudaFuncSetAttribute(lt::lazy_ratio_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              lt::RatioLayout<64>::bytes(lt::kRatioMaxGroup * 256)) != cudaSuccess ||
@@ -107,23 +111,37 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 extern "C" {
 
-lt_status lt_prefill_attn(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O, float* LSE,
-                          float softmax_scale, lt_stream stream) {
+// Shared by lt_prefill_attn and lt_prefill_attn_ratio: checks, descriptors,
+// launch.  `ratio` null selects the plain attention kernel.
+static lt_status launch_attention(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
+                                  float* LSE, float softmax_scale, int S, int W, int n_obs, float* ratio,
+                                  lt_stream stream) {
   lt_status st = check_shape(shape);
   if (st != LT_OK) return st;
   if (!std::isfinite(softmax_scale)) return LT_ERR_INVALID_ARG;
+  if (ratio && (!aligned(ratio, 4) || S < 0 || W < 0 || (long long)S + W < 1 || n_obs < 1 || n_obs > 4096))
+    return LT_ERR_INVALID_ARG;
   const int T = shape->total_tokens;
   const int max_len = shape->cu_seqlens ? shape->max_seqlen : T;
-  if (T == 0) return LT_OK;  // nothing to read or write; the pointers may be null
-  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || !aligned(LSE, 4))
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T > 0 && (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || !aligned(LSE, 4)))
     return LT_ERR_INVALID_ARG;
-  if (max_len == 0) return LT_OK;
-  const long long n_qtiles = (max_len + 127) / 128;
-  const long long num_tiles = n_qtiles * shape->batch * shape->hq;
-  if (num_tiles > INT_MAX) return LT_ERR_INVALID_ARG;
-
   DeviceInfo* dev = nullptr;
-  if ((st = device_info(&dev)) != LT_OK) return st;
+  if (ratio) {
+    // The kernel adds each tile's share of the mean; sequences without tokens keep 0.
+    if ((st = device_info(&dev)) != LT_OK) return st;
+    if (cudaMemsetAsync(ratio, 0, sizeof(float) * size_t(shape->batch) * shape->hq, s) != cudaSuccess)
+      return LT_ERR_CUDA;
+  }
+  if (T == 0 || max_len == 0) return LT_OK;  // nothing to read or write
+  const int group = shape->hq / shape->hkv;
+  const long long n_qtiles = (max_len + 127) / 128;
+  const bool pair_heads = (group % 2) == 0;
+  const long long num_items = pair_heads ? n_qtiles * shape->batch * (shape->hq / 2)
+                                         : ((n_qtiles + 1) / 2) * shape->batch * shape->hq;
+  if (num_items > INT_MAX) return LT_ERR_INVALID_ARG;
+
+  if (!dev && (st = device_info(&dev)) != LT_OK) return st;
   const int d = shape->head_dim;
   CUtensorMap mq, mk, mv;
   if (make_map(&mq, Q, d, shape->hq, T) != LT_OK || make_map(&mk, K, d, shape->hkv, T) != LT_OK ||
@@ -135,20 +153,46 @@ lt_status lt_prefill_attn(const lt_shape* shape, const void* Q, const void* K, c
   p.total_tokens = T;
   p.hq = shape->hq;
   p.hkv = shape->hkv;
+  p.group = group;
   p.n_qtiles = int(n_qtiles);
-  p.num_tiles = int(num_tiles);
+  p.pair_heads = pair_heads ? 1 : 0;
+  p.num_items = int(num_items);
   p.cu_seqlens = shape->cu_seqlens;
   p.O = static_cast<__nv_bfloat16*>(O);
   p.LSE = LSE;
   p.scale_log2 = resolve_scale(softmax_scale, d) * kLog2e;
   p.status = dev->status;
-  const int grid = int(num_tiles < dev->sm_count ? num_tiles : dev->sm_count);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    lt::attn_fwd_kernel<64><<<grid, lt::AttnLayout<64>::kThreads, lt::AttnLayout<64>::kAlloc, s>>>(mq, mk, mv, p);
-  else
-    lt::attn_fwd_kernel<128><<<grid, lt::AttnLayout<128>::kThreads, lt::AttnLayout<128>::kAlloc, s>>>(mq, mk, mv, p);
+  p.ratio = ratio;
+  p.S = S;
+  p.W = W;
+  p.n_obs = n_obs;
+  const int grid = int(num_items < dev->sm_count ? num_items : dev->sm_count);
+  if (d == 64) {
+    constexpr int kThreads = lt::AttnLayout<64>::kThreads, kSmem = lt::AttnLayout<64>::kAlloc;
+    if (ratio)
+      lt::attn_fwd_kernel<64, true><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
+    else
+      lt::attn_fwd_kernel<64, false><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
+  } else {
+    constexpr int kThreads = lt::AttnLayout<128>::kThreads, kSmem = lt::AttnLayout<128>::kAlloc;
+    if (ratio)
+      lt::attn_fwd_kernel<128, true><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
+    else
+      lt::attn_fwd_kernel<128, false><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
+  }
   return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_prefill_attn(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O, float* LSE,
+                          float softmax_scale, lt_stream stream) {
+  return launch_attention(shape, Q, K, V, O, LSE, softmax_scale, 0, 0, 0, nullptr, stream);
+}
+
+lt_status lt_prefill_attn_ratio(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
+                                float* LSE, float softmax_scale, int S, int W, int n_obs, float* ratio,
+                                lt_stream stream) {
+  if (!ratio) return LT_ERR_INVALID_ARG;
+  return launch_attention(shape, Q, K, V, O, LSE, softmax_scale, S, W, n_obs, ratio, stream);
 }
 
 lt_status lt_lazy_ratio(const lt_shape* shape, const void* Q, const void* K, const float* LSE, float softmax_scale,

@@ -139,6 +139,19 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]: A (M x K, K-major) is read from tensor memory,
+// lane m = row m, each 32-bit column holding two consecutive K elements (the
+// lower one in the low half).  Issued by a single thread.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrives (once) on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -197,8 +210,29 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// 16 consecutive 32-bit TMEM columns of this thread's lane (32x32b shape).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Warpgroup register split (all 128 threads of an aligned warpgroup execute it).
+// The counts must fit the block's launch allocation (threads x launch registers).
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 // --------------------------------------------------------------------- misc
 
@@ -206,6 +240,26 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x evaluated on the FMA pipe instead of the MUFU unit, to share the
+// exponentials of the softmax between the two.  Base-2 range reduction:
+// x = n + f with n = round(x) (the 1.5 * 2^23 shift leaves n in the low mantissa
+// bits) and f in [-1/2, 1/2]; 2^f by a cubic fitted here for relative error on
+// [-1/2, 1/2] (Lawson's iteratively reweighted least squares over Chebyshev
+// points; max relative error 7.5e-5 in fp32, below bf16 rounding of P); 2^n is
+// added to the exponent field.  x is clamped at -126 so the exponent stays in
+// range (2^-126 is zero for the softmax sums).
+__device__ __forceinline__ float exp2_fma(float x) {
+  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
+  constexpr float kC2 = 0.2426111400127411f, kC3 = 0.0551716685295105f;
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  x = fmaxf(x, -126.f);
+  const float t = x + kShift;
+  const uint32_t n_bits = __float_as_uint(t) << 23;
+  const float f = x - (t - kShift);
+  const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
+  return __uint_as_float(__float_as_uint(p) + n_bits);
 }
 
 __device__ __forceinline__ float fast_log2(float x) {

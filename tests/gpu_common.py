@@ -26,6 +26,11 @@ def gpu_attention(cfg, Q, K, V):
     return lt.lt_prefill_attn(Q, K, V, cu_seqlens=cu, max_seqlen=cfg.max_seqlen)
 
 
+def gpu_fused(cfg, Q, K, V):
+    cu = cu_tensor(cfg) if cfg.batch > 1 else None
+    return lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, cu_seqlens=cu, max_seqlen=cfg.max_seqlen)
+
+
 def gpu_ratio(cfg, Q, K, LSE):
     cu = cu_tensor(cfg) if cfg.batch > 1 else None
     return lt.lt_lazy_ratio(Q, K, LSE, cfg.S, cfg.W, cfg.n_obs, cu_seqlens=cu, max_seqlen=cfg.max_seqlen)
