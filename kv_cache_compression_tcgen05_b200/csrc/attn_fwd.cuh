@@ -14,10 +14,13 @@
 //   * warp-specialised, 10 warps:
 //       warp 0      TMA producer: the item's two Q tiles (double buffered) and
 //                   a ring of K/V tiles (128 keys x d, 128-byte swizzle);
-//       warp 1      owns the TMEM allocation; one thread issues every tcgen05.mma
-//                   in the order  PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), ...
-//                   so the tensor core works for one tile while the other
-//                   tile's softmax runs;
+//       warp 1      owns the TMEM allocation; one thread issues every
+//                   tcgen05.mma in the order
+//                       S_A(0), S_B(0), [PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)]
+//                   so the tensor core works on one tile while the other
+//                   tile's softmax runs (shared-memory descriptors are built
+//                   once and advanced by address/16, so the single issuing
+//                   thread spends little per instruction);
 //       warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: thread =
 //                   query row = TMEM lane.  tcgen05.ld of the 128 scores, causal
 //                   mask on the diagonal tile, running max in the log2 domain
@@ -26,16 +29,12 @@
 //                   exp2, bf16 P written back over the scores in TMEM with
 //                   tcgen05.st (P is the A operand of O += P V, read from TMEM);
 //                   epilogue O / l and LSE = (m + log2 l) ln 2, written once.
-//   * d = 128, TMEM [0,128) S/P of A, [128,256) S/P of B, [256,384) O of A,
-//     [384,512) O of B.  P overwrites the first half of its S columns; the MMAs
-//     of one thread execute in issue order, so S_X(j+1), issued after PV_X(j),
-//     never overwrites P_X(j) before PV_X(j) has read it, and once S_X(j+1) is
-//     complete so is PV_X(j): the softmax may rescale O_X right away.
-//   * d = 64, TMEM S [0,128) [128,256), P [256,320) [320,384), O [384,448)
-//     [448,512).  With P in its own columns the softmax frees S as soon as the
-//     scores are in registers, and S_X(j+1) runs on the tensor core while the
-//     softmax of tile j is still exponentiating; the softmax waits for PV_X(j-1)
-//     only before it overwrites P and rescales O.
+//   * TMEM columns: [0,128) S/P of A, [128,256) S/P of B, [256,256+d) O of A,
+//     [256+d, 256+2d) O of B.  P overwrites the first half of its S columns.
+//     The MMAs of one thread execute in issue order, so S_X(j+1), issued after
+//     PV_X(j), never overwrites P_X(j) before PV_X(j) has read it, and once
+//     S_X(j+1) is complete so is PV_X(j): the softmax may rescale O_X as soon
+//     as it sees S_X(j+1).
 //
 // Fused lazy ratio (press-release page, "LightTransfer方法详解": attention
 // weights from the query to the initial and the recent keys): for the last
@@ -82,20 +81,13 @@ struct AttnLayout {
   static constexpr int kQOff = 0;                     // [2 buffers][2 tiles]
   static constexpr int kRingOff = kQOff + 4 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 + 2 + 2 * kStages + 2 + 2 + 2 + 2 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 64;
   static constexpr int kAlloc = kBytes + 1024;        // room to align the base to 1024 B
   static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 512;
-  // d = 64: P of each tile has its own 64 columns, so S(j+1) may be written while
-  // P(j) waits for its MMA: S [0,128) [128,256), P [256,320) [320,384),
-  // O [384,448) [448,512).  d = 128: P overwrites the first half of its S
-  // columns: S/P [0,128) [128,256), O [256,384) [384,512).
-  static constexpr bool kSepP = D == 64;
-  static constexpr uint32_t kTmemP = kSepP ? 256 : 0;
-  static constexpr uint32_t kPStride = kSepP ? 64 : 128;
-  static constexpr uint32_t kTmemO = kSepP ? 384 : 256;
+  static constexpr uint32_t kTmemO = 256;
 };
 
 struct AttnItem {
@@ -167,17 +159,11 @@ __device__ __forceinline__ int attn_item_index(int round, int cta, int grid) {
 // Every kEmuPeriod-th pair of softmax columns takes the FMA-pipe exp2 (0: none).
 constexpr int kEmuPeriod = 0;
 
-template <bool V>
-struct BoolConst {
-  static constexpr bool value = V;
-};
-
 template <int D, bool kRatio>
 __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using Lay = AttnLayout<D>;
-  constexpr bool kSepP = Lay::kSepP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + Lay::kQOff;
@@ -191,9 +177,7 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
   uint64_t* p_full = s_full + 2;                 // [2 tiles]     softmax -> MMA (128 arrivals)
   uint64_t* o_full = p_full + 2;                 // [2 tiles]     MMA -> epilogue
   uint64_t* o_empty = o_full + 2;                // [2 tiles]     epilogue -> MMA (128 arrivals)
-  uint64_t* s_free = o_empty + 2;                // [2 tiles]     softmax -> MMA (128 arrivals; d = 64)
-  uint64_t* pv_done = s_free + 2;                // [2 tiles]     MMA -> softmax (d = 64)
-  uint64_t* drain = pv_done + 2;                 // [1]           MMA drain on abort
+  uint64_t* drain = o_empty + 2;                 // [1]           MMA drain on abort
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
   // Never raised: the drain waits after an abort end on completion or time only.
@@ -214,14 +198,12 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
       mbar_init(&p_full[i], 128);
       mbar_init(&o_full[i], 1);
       mbar_init(&o_empty[i], 128);
-      mbar_init(&s_free[i], 128);
-      mbar_init(&pv_done[i], 1);
     }
+    mbar_init(drain, 1);
     for (int i = 0; i < Lay::kStages; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(drain, 1);
     *abort_flag = 0;
     *no_abort = 0;
     ratio_cnt[0] = ratio_cnt[1] = 0;
@@ -285,9 +267,14 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
+      // Shared-memory descriptors differ only in the start-address field
+      // (address / 16, 14 bits; the shared window is below 256 KB): built once,
+      // advanced by byte offset / 16 per MMA.
+      const uint64_t q_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t k_desc = smem_desc_sw128(smem_u32(sRing), 16, 1024);
+      const uint64_t v_desc = smem_desc_sw128(smem_u32(sRing), Lay::kSub, 1024);
       int ring = 0, nq = 0;
       int cnt_p0 = 0, cnt_p1 = 0;   // P tiles consumed, per tile slot
-      int cnt_s0 = 0, cnt_s1 = 0;   // S tiles issued, per tile slot (d = 64)
       int cnt_o0 = 0, cnt_o1 = 0;   // items finished, per tile slot
       bool ok = true;
       for (int round = 0; ok && round * grid < p.num_items; ++round) {
@@ -300,28 +287,22 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
         const int base = ring;
         const int n = it.n[0];
         const int nB = it.hasB ? it.n[1] : 0;
+        ring = base + 2 * n;
         auto slot_of = [&](int j, int kv) { return (base + 2 * j + kv) % Lay::kStages; };
         auto phase_of = [&](int j, int kv) { return ((base + 2 * j + kv) / Lay::kStages) & 1; };
         // S_x(j) = Q_x K_j^T into the tile's TMEM score columns.
         auto issue_s = [&](int x, int j) -> bool {
           const int slot = slot_of(j, 0);
-          if constexpr (kSepP) {
-            // The softmax must have loaded the previous scores of this tile.
-            int& cnt_s = x ? cnt_s1 : cnt_s0;
-            if (cnt_s > 0 && !mbar_wait(&s_free[x], (cnt_s - 1) & 1, ctl)) return false;
-            ++cnt_s;
-          }
           if (x == 0) {   // tile A always uses K_j first
             if (!mbar_wait(&kv_full[slot], phase_of(j, 0), ctl)) return false;
           }
           tc_fence_after();
-          const uint32_t q_addr = smem_u32(sQ + (qb * 2 + x) * Lay::kTileBytes);
-          const uint32_t k_addr = smem_u32(sRing + slot * Lay::kTileBytes);
+          const uint64_t qd = q_desc + uint64_t(((qb * 2 + x) * Lay::kTileBytes) >> 4);
+          const uint64_t kd = k_desc + uint64_t((slot * Lay::kTileBytes) >> 4);
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k >> 2) * Lay::kSub + (k & 3) * 32;
-            mma_bf16_ss(tmem + x * 128, smem_desc_sw128(q_addr + off, 16, 1024),
-                        smem_desc_sw128(k_addr + off, 16, 1024), kIdS, k > 0 ? 1u : 0u);
+            const uint32_t off16 = ((k >> 2) * Lay::kSub + (k & 3) * 32) >> 4;
+            mma_bf16_ss(tmem + x * 128, qd + off16, kd + off16, kIdS, k > 0 ? 1u : 0u);
           }
           mma_commit(&s_full[x]);
           const bool last_use = x == 1 || j >= nB;
@@ -339,14 +320,12 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
           const int slot = slot_of(j, 1);
           if (x == 0 && !mbar_wait(&kv_full[slot], phase_of(j, 1), ctl)) return false;
           tc_fence_after();
-          const uint32_t v_addr = smem_u32(sRing + slot * Lay::kTileBytes);
+          const uint64_t vd = v_desc + uint64_t((slot * Lay::kTileBytes) >> 4);
+          const uint32_t o_tmem = tmem + Lay::kTmemO + x * D;
 #pragma unroll
-          for (int k = 0; k < 128 / 16; ++k) {
-            const uint64_t b = smem_desc_sw128(v_addr + k * 2048, Lay::kSub, 1024);
-            mma_bf16_ts(tmem + Lay::kTmemO + x * D, tmem + Lay::kTmemP + x * Lay::kPStride + k * 8, b, kIdPV,
+          for (int k = 0; k < 128 / 16; ++k)
+            mma_bf16_ts(o_tmem, tmem + x * 128 + k * 8, vd + uint64_t((k * 2048) >> 4), kIdPV,
                         (j > 0 || k > 0) ? 1u : 0u);
-          }
-          if constexpr (kSepP) mma_commit(&pv_done[x]);
           const bool last_use = x == 1 || j >= nB;
           if (last_use) mma_commit(&kv_empty[slot]);
           if ((x == 0 && j == n - 1) || (x == 1 && j == nB - 1)) {
@@ -357,22 +336,10 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
         };
 
         ok = issue_s(0, 0) && (nB == 0 || issue_s(1, 0));
-        if constexpr (kSepP) {
-          // S(j+1) as soon as the softmax has read S(j); PV(j) once P(j) is written.
-          for (int j = 0; ok && j < n; ++j) {
-            if (j + 1 < n) ok = issue_s(0, j + 1);
-            if (ok && j + 1 < nB) ok = issue_s(1, j + 1);
-            if (ok) ok = issue_pv(0, j);
-            if (ok && j < nB) ok = issue_pv(1, j);
-          }
-        } else {
-          // P(j) overwrites S(j): PV(j) must be issued before S(j+1).
-          for (int j = 0; ok && j < n; ++j) {
-            ok = issue_pv(0, j) && (j + 1 >= n || issue_s(0, j + 1));
-            if (ok && j < nB) ok = issue_pv(1, j) && (j + 1 >= nB || issue_s(1, j + 1));
-          }
+        for (int j = 0; ok && j < n; ++j) {
+          ok = issue_pv(0, j) && (j + 1 >= n || issue_s(0, j + 1));
+          if (ok && j < nB) ok = issue_pv(1, j) && (j + 1 >= nB || issue_s(1, j + 1));
         }
-        ring = base + 2 * n;
       }
       if (!ok) {
         mma_commit(drain);
@@ -386,7 +353,6 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
     const int row = wq * 32 + lane;            // query row within the tile
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const uint32_t s_col = tmem + lane_off + x * 128;
-    const uint32_t p_col = tmem + lane_off + Lay::kTmemP + x * Lay::kPStride;
     const uint32_t o_col = tmem + lane_off + Lay::kTmemO + x * D;
     const float sl2 = p.scale_log2;
     int cnt_s = 0, cnt_o = 0;
@@ -432,11 +398,6 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
           tmem_ld32(s_col + 96, c3);
           tmem_wait_ld();
         }
-        if constexpr (kSepP) {
-          // The scores are in registers: the MMA may overwrite S with S(j+1).
-          tc_fence_before();
-          mbar_arrive(&s_free[x]);
-        }
         if (diag) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
@@ -459,65 +420,60 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
         }
         l_run *= alpha;
         if constexpr (kRatio) num *= alpha;
-        if constexpr (kSepP) {
-          // P(j) reuses the P columns and O(j) accumulates onto O: both need PV(j-1) done.
-          if (cnt_s > 1) {   // cnt_s - 1 = index of this tile among the slot's tiles
-            ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], (cnt_s - 2) & 1, ctl));
-            if (!ok) break;
-            tc_fence_after();
-          }
-        }
         // exp2 in 32-column chunks; each chunk's bf16 P goes to TMEM (16
         // columns) as soon as it is packed.  Every kEmuPeriod-th pair of
         // columns may use the FMA-pipe exp2 to share work with the MUFU unit.
         float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         const float neg_m = -m_run;
-        float racc = 0.f;
-        bool band = false;
-        int win_lo = 0;
-        if constexpr (kRatio) {
-          win_lo = qpos - p.W + 1;
-          band = row_obs && (j * 128 < p.S || j * 128 + 127 >= win_lo);
-        }
-        auto exp_chunks = [&](auto with_band) {
-          constexpr bool kBand = decltype(with_band)::value;
 #pragma unroll
-          for (int cb = 0; cb < 4; ++cb) {
-            uint32_t pk[16];
+        for (int cb = 0; cb < 4; ++cb) {
+          uint32_t pk[16];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const int c0 = cb * 32 + 2 * c;
-              const float x0 = fmaf(__uint_as_float(sr[c0]), sl2, neg_m);
-              const float x1 = fmaf(__uint_as_float(sr[c0 + 1]), sl2, neg_m);
-              float p0, p1;
-              if (kEmuPeriod > 0 && (c % kEmuPeriod) == kEmuPeriod - 1) {
-                p0 = exp2_fma(x0);
-                p1 = exp2_fma(x1);
-              } else {
-                p0 = fast_exp2(x0);
-                p1 = fast_exp2(x1);
-              }
-              sum8[c & 7] += p0 + p1;
-              pk[c] = pack_bf16x2(p0, p1);
-              if constexpr (kBand) {
-                // Weights of the sink keys and the W most recent keys of this row.
-                const int k0 = j * 128 + c0, k1 = k0 + 1;
-                racc += (k0 <= qpos && (k0 < p.S || k0 >= win_lo)) ? p0 : 0.f;
-                racc += (k1 <= qpos && (k1 < p.S || k1 >= win_lo)) ? p1 : 0.f;
-              }
+          for (int c = 0; c < 16; ++c) {
+            const int c0 = cb * 32 + 2 * c;
+            const float x0 = fmaf(__uint_as_float(sr[c0]), sl2, neg_m);
+            const float x1 = fmaf(__uint_as_float(sr[c0 + 1]), sl2, neg_m);
+            float p0, p1;
+            constexpr int kPeriod = kEmuPeriod > 0 ? kEmuPeriod : 1;
+            if (kEmuPeriod > 0 && (c % kPeriod) == kPeriod - 1) {
+              p0 = exp2_fma(x0);
+              p1 = exp2_fma(x1);
+            } else {
+              p0 = fast_exp2(x0);
+              p1 = fast_exp2(x1);
             }
-            tmem_st16(p_col + cb * 16, pk);
+            sum8[c & 7] += p0 + p1;
+            pk[c] = pack_bf16x2(p0, p1);
           }
-        };
-        if (kRatio && __any_sync(0xffffffffu, band))
-          exp_chunks(BoolConst<true>{});
-        else
-          exp_chunks(BoolConst<false>{});
-        l_run += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
-        if constexpr (kRatio) num += band ? racc : 0.f;
+          tmem_st16(s_col + cb * 16, pk);
+        }
+        const float tile_sum =
+            ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+        l_run += tile_sum;
+        if constexpr (kRatio) {
+          // Weights of the keys in K_i = [0, min(S, i+1)) U [max(S, i-W+1), i]
+          // within this key tile (columns c = key - 128 j).  Keys after i carry
+          // weight 0 (causal mask), so a tile that starts inside the window
+          // counts whole; only the tile holding the window's first key and the
+          // tile holding the sinks need a per-key mask.
+          const int win_c = qpos - p.W + 1 - j * 128;   // first window column
+          const int sink_c = p.S - j * 128;              // columns below it are sinks
+          const bool whole = row_obs && win_c <= 0;
+          const bool part = row_obs && !whole && (win_c < 128 || sink_c > 0);
+          if (whole) num += tile_sum;
+          if (__any_sync(0xffffffffu, part)) {
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+              const float w = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, neg_m));
+              acc += (c < sink_c || c >= win_c) ? w : 0.f;
+            }
+            if (part) num += acc;
+          }
+        }
         if (j > 0 && __any_sync(0xffffffffu, need)) {
-          // PV(j-1) is complete (d = 128: S(j) was issued after it; d = 64: waited
-          // on above): rescale O in TMEM before PV(j) accumulates onto it.
+          // PV(j-1) is complete (S(j) was issued after it by the same thread):
+          // rescale O in TMEM before PV(j) accumulates onto it.
 #pragma unroll
           for (int cb = 0; cb < D / 32; ++cb) {
             uint32_t o[32];
