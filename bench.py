@@ -63,7 +63,7 @@ def source_digest(paths):
 def recorded_traffic(config_name):
     """DRAM bytes per attention launch from the committed ncu summary, or None if
     the kernel source changed since the counters were taken."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_{config_name}.traffic.json")
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{config_name}.traffic.txt")
     if not os.path.exists(path):
         return None
     with open(path) as f:
@@ -159,10 +159,11 @@ def dist_setup(n_gpus):
     return rank, world, local
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """Largest value over all ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 

@@ -190,6 +190,15 @@ lt_status lt_compact_kv(const lt_shape* shape, const void* K, const void* V, con
  */
 lt_status lt_device_status(int clear);
 
+/*
+ * Self-test of the kernels' bounded waits: enqueues a one-thread kernel that
+ * waits, with the same wait routine the kernels use, on an mbarrier nothing
+ * arrives on; after limit_us microseconds (1 .. 10^7) it gives up, sets the
+ * device status word and returns.  A following lt_device_status reports
+ * LT_ERR_TIMEOUT; the device and the context stay usable.
+ */
+lt_status lt_selftest_wait_timeout(unsigned limit_us, lt_stream stream);
+
 /* Human-readable name of a status. */
 const char* lt_status_string(lt_status status);
 

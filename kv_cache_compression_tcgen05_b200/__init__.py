@@ -30,6 +30,7 @@ from .binding import (  # noqa: F401
     lt_queue_push,
     lt_queue_size,
     lt_select_layers,
+    lt_selftest_wait_timeout,
     lt_status_string,
     lt_version,
     LayerQueue,

@@ -56,6 +56,7 @@ _SIGS = {
     "lt_queue_destroy": (None, [_vp]),
     "lt_compact_kv": (_i, [_shp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp]),
     "lt_device_status": (_i, [_i]),
+    "lt_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "lt_status_string": (ctypes.c_char_p, [_i]),
     "lt_version": (_i, []),
 }
@@ -314,3 +315,8 @@ class LayerQueue:
 def lt_device_status(clear: bool = True) -> int:
     """LT_OK or LT_ERR_TIMEOUT (synchronises the current device)."""
     return library().lt_device_status(1 if clear else 0)
+
+
+def lt_selftest_wait_timeout(limit_us, stream=None):
+    """Run the bounded-wait self-test kernel (see include/lt.h)."""
+    _check(library().lt_selftest_wait_timeout(int(limit_us), _stream_handle(stream)), "lt_selftest_wait_timeout")

@@ -11,7 +11,7 @@
 //     read the same K/V stream: two query heads of one KV head at the same
 //     q-tile when the GQA group is even, otherwise two consecutive q-tiles of
 //     one head (the earlier tile then skips the last key tile).
-//   * warp-specialised, 10 warps:
+//   * warp-specialised, 10 working warps (12 launched):
 //       warp 0      TMA producer: the item's two Q tiles (double buffered) and
 //                   a ring of K/V tiles (128 keys x d, 128-byte swizzle);
 //       warp 1      owns the TMEM allocation; one thread issues every
@@ -85,7 +85,9 @@ struct AttnLayout {
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 64;
   static constexpr int kAlloc = kBytes + 1024;        // room to align the base to 1024 B
-  static constexpr int kThreads = 320;
+  // 10 working warps; two more idle warps make ptxas allocate the softmax
+  // path without spills (same 168 registers per thread either way).
+  static constexpr int kThreads = 384;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemO = 256;
 };
@@ -155,9 +157,6 @@ __device__ __forceinline__ bool attn_decode(const AttnParams& p, int t, AttnItem
 __device__ __forceinline__ int attn_item_index(int round, int cta, int grid) {
   return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
 }
-
-// Every kEmuPeriod-th pair of softmax columns takes the FMA-pipe exp2 (0: none).
-constexpr int kEmuPeriod = 0;
 
 template <int D, bool kRatio>
 __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
@@ -346,7 +345,7 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
         mbar_wait(drain, 0, drain_ctl);
       }
     }
-  } else {
+  } else if (warp < 10) {
     // --------------------------------------------------------------- softmax
     const int x = (warp - 2) >> 2;             // tile slot: 0 = A (warps 2..5), 1 = B (warps 6..9)
     const int wq = warp & 3;                   // TMEM lane quarter of this warp
@@ -403,14 +402,16 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
           for (int c = 0; c < 128; ++c)
             if (c > row) sr[c] = __float_as_uint(-INFINITY);
         }
-        // Row maximum as 8 independent chains.
+        // Row maximum: 8 independent chains of three-input max.
+        // Columns 0..15 seed the chains; c = 16, 32, ..., 112 covers 16..127.
         float mx8[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = __uint_as_float(sr[k]);
+        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[8 + k]));
 #pragma unroll
-        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int c = 16; c < 128; c += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool need = m_new > m_run + 8.f;
         float alpha = 1.f;
@@ -421,8 +422,7 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
         l_run *= alpha;
         if constexpr (kRatio) num *= alpha;
         // exp2 in 32-column chunks; each chunk's bf16 P goes to TMEM (16
-        // columns) as soon as it is packed.  Every kEmuPeriod-th pair of
-        // columns may use the FMA-pipe exp2 to share work with the MUFU unit.
+        // columns) as soon as it is packed.
         float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         const float neg_m = -m_run;
 #pragma unroll
@@ -433,15 +433,8 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
             const int c0 = cb * 32 + 2 * c;
             const float x0 = fmaf(__uint_as_float(sr[c0]), sl2, neg_m);
             const float x1 = fmaf(__uint_as_float(sr[c0 + 1]), sl2, neg_m);
-            float p0, p1;
-            constexpr int kPeriod = kEmuPeriod > 0 ? kEmuPeriod : 1;
-            if (kEmuPeriod > 0 && (c % kPeriod) == kPeriod - 1) {
-              p0 = exp2_fma(x0);
-              p1 = exp2_fma(x1);
-            } else {
-              p0 = fast_exp2(x0);
-              p1 = fast_exp2(x1);
-            }
+            const float p0 = fast_exp2(x0);
+            const float p1 = fast_exp2(x1);
             sum8[c & 7] += p0 + p1;
             pk[c] = pack_bf16x2(p0, p1);
           }

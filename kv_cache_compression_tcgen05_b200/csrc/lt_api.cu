@@ -14,6 +14,7 @@
 #include "attn_fwd.cuh"
 #include "compact_kv.cuh"
 #include "lazy_ratio.cuh"
+#include "selftest.cuh"
 #include "lt.h"
 
 namespace {
@@ -282,6 +283,16 @@ lt_status lt_compact_kv(const lt_shape* shape, const void* K, const void* V, con
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   lt::compact_kv_kernel<<<int(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_selftest_wait_timeout(unsigned limit_us, lt_stream stream) {
+  if (limit_us == 0 || limit_us > 10000000u) return LT_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  lt_status st = device_info(&dev);
+  if (st != LT_OK) return st;
+  lt::wait_timeout_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      dev->status, (unsigned long long)limit_us * 1000ull);
   return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
 }
 

@@ -61,10 +61,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 struct WaitCtl {
   volatile int* abort_flag;   // shared memory
   unsigned* status;           // global status word
+  unsigned long long limit_ns = kWaitLimitNs;
 };
 
 // Waits until the phase with the given parity has completed.  Returns false if
-// the CTA is aborting or the wait exceeded kWaitLimitNs (then it also raises the
+// the CTA is aborting or the wait exceeded ctl.limit_ns (then it also raises the
 // abort flag and the status word).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -73,7 +74,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     if (mbar_try_wait(bar, parity)) return true;
     if ((spin & 63u) == 0) {
       if (*ctl.abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > ctl.limit_ns) {
         *ctl.abort_flag = 1;
         atomicOr(ctl.status, kErrTimeout);
         return false;
@@ -242,24 +243,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x evaluated on the FMA pipe instead of the MUFU unit, to share the
-// exponentials of the softmax between the two.  Base-2 range reduction:
-// x = n + f with n = round(x) (the 1.5 * 2^23 shift leaves n in the low mantissa
-// bits) and f in [-1/2, 1/2]; 2^f by a cubic fitted here for relative error on
-// [-1/2, 1/2] (Lawson's iteratively reweighted least squares over Chebyshev
-// points; max relative error 7.5e-5 in fp32, below bf16 rounding of P); 2^n is
-// added to the exponent field.  x is clamped at -126 so the exponent stays in
-// range (2^-126 is zero for the softmax sums).
-__device__ __forceinline__ float exp2_fma(float x) {
-  constexpr float kC0 = 0.9999280571937561f, kC1 = 0.6932609677314758f;
-  constexpr float kC2 = 0.2426111400127411f, kC3 = 0.0551716685295105f;
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  x = fmaxf(x, -126.f);
-  const float t = x + kShift;
-  const uint32_t n_bits = __float_as_uint(t) << 23;
-  const float f = x - (t - kShift);
-  const float p = fmaf(fmaf(fmaf(kC3, f, kC2), f, kC1), f, kC0);
-  return __uint_as_float(__float_as_uint(p) + n_bits);
+// max(a, b, c) in one instruction (three-input max of sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ float fast_log2(float x) {
