@@ -4,14 +4,14 @@
 
 One step is one pass of the whole path over one prefill of the workload: for
 every layer the causal GQA attention with its LSE fused with the lazy ratio
-(lt_prefill_attn_ratio), the layer priority queue (lt_queue_push, host) and,
-for each layer the queue demotes, the KV compaction (lt_compact_kv).  The plain
-attention (lt_prefill_attn) and the separate ratio pass from the LSE
-(lt_lazy_ratio) are timed beside it for the ratio-overhead figures.  The
-per-layer Q/K/V of all layers are resident in HBM before timing (together far
-larger than the 126 MB L2, so no L2 flush is needed between steps).  The ratio
-of layer l is read back asynchronously and pushed while layer l+1's attention
-runs, so the queue never stalls the GPU.
+(lt_prefill_attn_ratio), the push of the layer's ratios into the device-resident
+layer queue (lt_dqueue_push) and the compaction of the layer the queue demotes,
+if any (lt_compact_kv_pending).  The whole step is one CUDA graph (no host round
+trip).  The per-layer Q/K/V of all layers are resident in HBM before timing
+(together far larger than the 126 MB L2, so no L2 flush is needed).  The plain
+attention (lt_prefill_attn), the separate ratio pass from the LSE
+(lt_lazy_ratio), the host queue and compaction (lt_compact_kv) are timed beside
+it.
 
 Rank 0 prints one JSON line.  With --gpus N > 1 (torchrun) every rank runs an
 independent replica of the workload (the path has no exchange step): weak
@@ -185,67 +185,40 @@ class Prefill:
         self.cu = torch.tensor(cfg.cu_seqlens(), dtype=torch.int32, device=device) if cfg.batch > 1 else None
         self.O = torch.empty((T, H, d), dtype=torch.bfloat16, device=device)
         self.LSE = torch.empty((H, T), dtype=torch.float32, device=device)
-        self.ratio_dev = torch.empty((cfg.layers, cfg.batch, H), dtype=torch.float32, device=device)
-        self.ratio_host = torch.empty((cfg.layers, cfg.batch, H), dtype=torch.float32, pin_memory=True)
+        self.ratio = torch.empty((cfg.layers, cfg.batch, H), dtype=torch.float32, device=device)
         slots = cfg.S + cfg.W
-        self.ks = torch.empty((cfg.budget, cfg.batch, cfg.hkv, slots, d), dtype=torch.bfloat16, device=device)
-        self.vs = torch.empty_like(self.ks)
-        self.slen = torch.empty((cfg.budget, cfg.batch), dtype=torch.int32, device=device)
-        self.masks = torch.zeros((cfg.layers, cfg.batch), dtype=torch.uint8, device=device)
-        self.mask_host = torch.zeros((cfg.layers, cfg.batch), dtype=torch.uint8, pin_memory=True)
-        self.events = [torch.cuda.Event() for _ in range(cfg.layers)]
-        self.launches = 0
-        self.attn_events = None
+        self.K_pool = torch.zeros((cfg.budget, cfg.batch, cfg.hkv, slots, d), dtype=torch.bfloat16, device=device)
+        self.V_pool = torch.zeros_like(self.K_pool)
+        self.pool_len = torch.zeros((cfg.budget, cfg.batch), dtype=torch.int32, device=device)
+        self.Kp = lt.layer_pointer_table([lay[1] for lay in self.layers])
+        self.Vp = lt.layer_pointer_table([lay[2] for lay in self.layers])
+        self.dq = lt.DeviceQueue(cfg.layers, cfg.budget, cfg.batch)
+        self.kw = dict(cu_seqlens=self.cu, max_seqlen=cfg.max_seqlen)
 
-    def step(self, time_kernels=False):
+    def enqueue_step(self, stream, events=None, layers=None):
+        """Enqueue one whole step on `stream`; `events` collects an (start, end)
+        pair of external timing events around every attention launch."""
         cfg, lt = self.cfg, self.lt
-        kw = dict(cu_seqlens=self.cu, max_seqlen=cfg.max_seqlen)
-        queues = [lt.LayerQueue(cfg.layers, cfg.budget) for _ in range(cfg.batch)]
-        demoted = []
-        self.launches = 0
-        ev = [] if time_kernels else None
-        mask_host = self.mask_host.numpy()
-        mask_host[:] = 0
-
-        def consume(l):
-            # Host side of layer l: its ratios are in pinned memory once its event fires.
-            self.events[l].synchronize()
-            newly = []
-            for b in range(cfg.batch):
-                d = queues[b].push(l, lt.lt_layer_score(self.ratio_host[l, b].numpy()))
-                if d >= 0:
-                    newly.append((d, b))
-            for d, b in newly:
-                mask_host[d, b] = 1
-            for d in sorted(set(x for x, _ in newly)):
-                k = len(demoted)
-                self.masks[d].copy_(self.mask_host[d], non_blocking=True)
-                Q, K, V = self.layers[d]
-                lt.lt_compact_kv(K, V, self.masks[d], cfg.S, cfg.W, k_stream=self.ks[k % cfg.budget],
-                                 v_stream=self.vs[k % cfg.budget], stream_len=self.slen[k % cfg.budget], **kw)
-                self.launches += 1
-                demoted.append(d)
-
+        layers = self.layers if layers is None else layers
+        lt.lt_dqueue_init(self.dq.state, cfg.layers, cfg.budget, cfg.batch, stream)
         for l in range(cfg.layers):
-            Q, K, V = self.layers[l]
-            if ev is not None:
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-            lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, out=self.O, lse=self.LSE,
-                                     ratio=self.ratio_dev[l], **kw)
-            if ev is not None:
-                e1.record()
-                ev.append((e0, e1))
-            self.launches += 1
-            self.ratio_host[l].copy_(self.ratio_dev[l], non_blocking=True)
-            self.events[l].record()
-            if l > 0:
-                consume(l - 1)
-        consume(cfg.layers - 1)
-        for q in queues:
-            q.close()
-        self.attn_events = ev
-        return demoted
+            Q, K, V = layers[l]
+            if events is not None:
+                e0 = torch.cuda.Event(enable_timing=True, external=True)
+                e1 = torch.cuda.Event(enable_timing=True, external=True)
+                e0.record(stream)
+            lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, out=self.O, lse=self.LSE, ratio=self.ratio[l],
+                                     stream=stream, **self.kw)
+            if events is not None:
+                e1.record(stream)
+                events.append((e0, e1))
+            lt.lt_dqueue_push(self.dq.state, cfg.layers, cfg.batch, l, self.ratio[l], stream)
+            lt.lt_compact_kv_pending(self.Kp, self.Vp, self.dq, cfg.S, cfg.W, self.K_pool, self.V_pool,
+                                     self.pool_len, cfg.total_tokens, cfg.hkv, cfg.d, stream=stream, **self.kw)
+
+    @staticmethod
+    def launches_per_step(cfg):
+        return 1 + 3 * cfg.layers   # queue init, then attention, push, compaction per layer
 
 
 def run_ours(args, cfg, rank, world):
@@ -253,30 +226,48 @@ def run_ours(args, cfg, rank, world):
     lt.library()
     peaks, peak_src = load_peaks()
     pf = Prefill(cfg, lt)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        pf.enqueue_step(stream)           # eager warm-up: per-device set-up happens outside capture
+    torch.cuda.synchronize()
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=stream):
+        pf.enqueue_step(stream)
+    g_timed = torch.cuda.CUDAGraph()
+    fused_ev = []
+    with torch.cuda.graph(g_timed, stream=stream):
+        for _ in range(args.steps):
+            pf.enqueue_step(stream, events=fused_ev)
     for _ in range(args.warmup):
-        pf.step()
+        g_step.replay()
     torch.cuda.synchronize()
     barrier(world)
 
-    # Device-timed region: K whole steps.
+    # Device-timed region: K whole steps (one graph replay).
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    fused_ev = []
     with ClockSampler(torch.cuda.current_device()) as clk:
-        torch.cuda.synchronize()
-        start.record()
-        launches = 0
-        for _ in range(args.steps):
-            pf.step(time_kernels=True)
-            launches += pf.launches
-            fused_ev += pf.attn_events
-        stop.record()
+        with torch.cuda.stream(stream):
+            torch.cuda.synchronize()
+            start.record(stream)
+            g_timed.replay()
+            stop.record(stream)
         torch.cuda.synchronize()
     barrier(world)
+    launches = args.steps * Prefill.launches_per_step(cfg)
     ms = max_over_ranks(start.elapsed_time(stop), world) / args.steps
     t_fused = statistics.mean(a.elapsed_time(b) for a, b in fused_ev) * 1e-3
+    # The demotions of the timed steps equal the host queue's on the same ratios.
+    mask_dev, order_dev = pf.dq.result()
+    host_order = []
+    for b in range(cfg.batch):
+        q = lt.LayerQueue(cfg.layers, cfg.budget)
+        r = pf.ratio.cpu().numpy()
+        host_order.append([x for x in (q.push(l, lt.lt_layer_score(r[l, b])) for l in range(cfg.layers)) if x >= 0])
+        q.close()
+    queue_agrees = all(order_dev[b].tolist() == host_order[b] for b in range(cfg.batch))
 
     # Beside the step: the plain attention and the separate ratio pass per layer.
-    kw = dict(cu_seqlens=pf.cu, max_seqlen=cfg.max_seqlen)
+    kw = pf.kw
     attn_ev, ratio_ev = [], []
     for rep in range(2):
         for l in range(cfg.layers):
@@ -285,7 +276,7 @@ def run_ours(args, cfg, rank, world):
             e0.record()
             lt.lt_prefill_attn(Q, K, V, out=pf.O, lse=pf.LSE, **kw)
             e1.record()
-            lt.lt_lazy_ratio(Q, K, pf.LSE, cfg.S, cfg.W, cfg.n_obs, out=pf.ratio_dev[l], **kw)
+            lt.lt_lazy_ratio(Q, K, pf.LSE, cfg.S, cfg.W, cfg.n_obs, out=pf.ratio[l], **kw)
             e2.record()
             if rep > 0:
                 attn_ev.append((e0, e1))
@@ -293,6 +284,7 @@ def run_ours(args, cfg, rank, world):
     torch.cuda.synchronize()
     t_attn = statistics.mean(a.elapsed_time(b) for a, b in attn_ev) * 1e-3
     t_ratio = statistics.mean(a.elapsed_time(b) for a, b in ratio_ev) * 1e-3
+
     if args.kernels_only:
         return {"metric": METRIC, "ms_per_step": round(ms, 4), "fused_us_per_layer": round(t_fused * 1e6, 2),
                 "attn_us_per_layer": round(t_attn * 1e6, 2), "ratio_us_per_layer": round(t_ratio * 1e6, 2),
@@ -308,8 +300,8 @@ def run_ours(args, cfg, rank, world):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             Q, K, V = pf.layers[l]
             e0.record()
-            lt.lt_compact_kv(K, V, mask1, cfg.S, cfg.W, k_stream=pf.ks[0], v_stream=pf.vs[0], stream_len=pf.slen[0],
-                             **kw)
+            lt.lt_compact_kv(K, V, mask1, cfg.S, cfg.W, k_stream=pf.K_pool[0], v_stream=pf.V_pool[0],
+                             stream_len=pf.pool_len[0], **kw)
             e1.record()
             torch.cuda.synchronize()
             if rep > 0:
@@ -349,6 +341,7 @@ def run_ours(args, cfg, rank, world):
             "layers": cfg.layers, "batch": cfg.batch, "seq_len": cfg.max_seqlen, "hq": cfg.hq, "hkv": cfg.hkv,
             "head_dim": cfg.d, "S": cfg.S, "W": cfg.W, "n_obs": cfg.n_obs, "budget": cfg.budget,
             "l2": "inputs of one step (all layers' Q/K/V) exceed L2; no flush between steps",
+            "step": "one CUDA graph: per layer fused attention+ratio, device queue push, device-driven compaction",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
         },
         "attn_tflops": round(achieved, 2),
@@ -361,6 +354,7 @@ def run_ours(args, cfg, rank, world):
         "separate_ratio_overhead_pct": round(100 * t_ratio / t_attn, 3),
         "compaction_gbs": round(comp_gbs, 1),
         "compaction_us_per_layer": round(t_comp * 1e6, 2),
+        "device_queue_matches_host_queue": queue_agrees,
         "roofline": {"kernel": "attn_fwd_kernel (fused with the lazy ratio)", "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": peak_sus, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_sus, 4), "traffic": traffic,
@@ -376,32 +370,34 @@ def run_ours(args, cfg, rank, world):
 def measure_e2e(args, cfg, lt, pf, world):
     """Same metric through the public calls with host buffers: every step copies
     each layer's Q/K/V from pinned host memory to the device and reads back each
-    layer's O and LSE, the ratios and the compacted KV, all inside the
-    device-timed region.  Uploads run on a side stream one layer ahead, read-backs
-    on another, so copies overlap the kernels.  The full K/V of every layer stay
-    on the device (the KV cache the queue manages); Q is double buffered."""
+    layer's O and LSE, the ratios and the streaming KV pool, all inside the
+    device-timed region.  Uploads run one layer ahead on a side stream and
+    read-backs on another, so copies overlap the kernels; the queue lives on the
+    device, so no step waits for the host.  The full K/V of every layer stay on
+    the device (the KV cache the queue manages); Q is double buffered."""
     host = [tuple(t.cpu().pin_memory() for t in lay) for lay in pf.layers]
     T, H, d = cfg.total_tokens, cfg.hq, cfg.d
     dev_q = [torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     dev_kv = [tuple(torch.empty_like(t) for t in lay[1:]) for lay in pf.layers]
+    Kp = lt.layer_pointer_table([kv[0] for kv in dev_kv])
+    Vp = lt.layer_pointer_table([kv[1] for kv in dev_kv])
     o_host = torch.empty((cfg.layers, T, H, d), dtype=torch.bfloat16, pin_memory=True)
     lse_host = torch.empty((cfg.layers, H, T), dtype=torch.float32, pin_memory=True)
-    ks_host = torch.empty(pf.ks.shape, dtype=torch.bfloat16, pin_memory=True)
+    ratio_host = torch.empty(pf.ratio.shape, dtype=torch.float32, pin_memory=True)
+    ks_host = torch.empty(pf.K_pool.shape, dtype=torch.bfloat16, pin_memory=True)
     vs_host = torch.empty_like(ks_host)
     O = [torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     LSE = [torch.empty((H, T), dtype=torch.float32, device="cuda") for _ in range(2)]
     copy_in, copy_out = torch.cuda.Stream(), torch.cuda.Stream()
     main = torch.cuda.current_stream()
-    kw = dict(cu_seqlens=pf.cu, max_seqlen=cfg.max_seqlen)
+    kw = pf.kw
     h2d = sum(t.numel() * t.element_size() for lay in host for t in lay)
-    d2h = (o_host.numel() * 2 + lse_host.numel() * 4 + pf.ratio_host.numel() * 4 + 2 * ks_host.numel() * 2)
+    d2h = o_host.numel() * 2 + lse_host.numel() * 4 + ratio_host.numel() * 4 + 2 * ks_host.numel() * 2
 
     def one_step():
         ready = [torch.cuda.Event() for _ in range(cfg.layers)]
         done = [torch.cuda.Event() for _ in range(cfg.layers)]
-        queues = [lt.LayerQueue(cfg.layers, cfg.budget) for _ in range(cfg.batch)]
-        n_dem = 0
-        mask_host = pf.mask_host.numpy()
+        computed = [torch.cuda.Event() for _ in range(cfg.layers)]
 
         def upload(l):
             with torch.cuda.stream(copy_in):
@@ -412,6 +408,7 @@ def measure_e2e(args, cfg, lt, pf, world):
                 dev_kv[l][1].copy_(host[l][2], non_blocking=True)
                 ready[l].record(copy_in)
 
+        lt.lt_dqueue_init(pf.dq.state, cfg.layers, cfg.budget, cfg.batch)
         upload(0)
         for l in range(cfg.layers):
             if l + 1 < cfg.layers:
@@ -419,39 +416,23 @@ def measure_e2e(args, cfg, lt, pf, world):
             main.wait_event(ready[l])
             Q, (K, V) = dev_q[l % 2], dev_kv[l]
             lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, out=O[l % 2], lse=LSE[l % 2],
-                                     ratio=pf.ratio_dev[l], **kw)
-            pf.ratio_host[l].copy_(pf.ratio_dev[l], non_blocking=True)
-            pf.events[l].record()
+                                     ratio=pf.ratio[l], **kw)
+            lt.lt_dqueue_push(pf.dq.state, cfg.layers, cfg.batch, l, pf.ratio[l])
+            lt.lt_compact_kv_pending(Kp, Vp, pf.dq, cfg.S, cfg.W, pf.K_pool, pf.V_pool, pf.pool_len, T, cfg.hkv, d,
+                                     **kw)
+            computed[l].record(main)
             with torch.cuda.stream(copy_out):
-                copy_out.wait_event(pf.events[l])
+                copy_out.wait_event(computed[l])
                 o_host[l].copy_(O[l % 2], non_blocking=True)
                 lse_host[l].copy_(LSE[l % 2], non_blocking=True)
                 done[l].record(copy_out)
-            pf.events[l].synchronize()
-            mask_host[l] = 0
-            dem = []
-            for b in range(cfg.batch):
-                m = queues[b].push(l, lt.lt_layer_score(pf.ratio_host[l, b].numpy()))
-                if m >= 0:
-                    dem.append((m, b))
-            for m in sorted(set(x for x, _ in dem)):
-                mask_host[m] = 0
-                for x, b in dem:
-                    if x == m:
-                        mask_host[m, b] = 1
-                pf.masks[m].copy_(pf.mask_host[m], non_blocking=True)
-                lt.lt_compact_kv(dev_kv[m][0], dev_kv[m][1], pf.masks[m], cfg.S, cfg.W,
-                                 k_stream=pf.ks[n_dem % cfg.budget], v_stream=pf.vs[n_dem % cfg.budget],
-                                 stream_len=pf.slen[n_dem % cfg.budget], **kw)
-                n_dem += 1
         with torch.cuda.stream(copy_out):
             copy_out.wait_stream(main)
-            ks_host.copy_(pf.ks, non_blocking=True)
-            vs_host.copy_(pf.vs, non_blocking=True)
+            ratio_host.copy_(pf.ratio, non_blocking=True)
+            ks_host.copy_(pf.K_pool, non_blocking=True)
+            vs_host.copy_(pf.V_pool, non_blocking=True)
         main.wait_stream(copy_out)
         main.wait_stream(copy_in)
-        for q in queues:
-            q.close()
 
     for _ in range(2):
         one_step()

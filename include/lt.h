@@ -48,6 +48,7 @@
 #ifndef LT_H_
 #define LT_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -182,6 +183,85 @@ void lt_queue_destroy(lt_queue* queue);
  */
 lt_status lt_compact_kv(const lt_shape* shape, const void* K, const void* V, const uint8_t* mask, int S, int W,
                         void* K_stream, void* V_stream, int32_t* stream_len, lt_stream stream);
+
+/*
+ * Device-resident layer queue (the queue of lt_queue_push kept in device
+ * memory, one per sequence of a batch), so that a whole prefill -- attention,
+ * ratio, queue, compaction for every layer -- is one stream of kernels with no
+ * host round trip (capturable in a CUDA graph).  Same rule and tie-break as
+ * lt_queue_push; the score is the mean of the layer's hq ratios computed exactly
+ * as lt_layer_score does, so host and device queues demote the same layers.
+ *
+ * state: caller-allocated device memory of lt_dqueue_state_bytes(L, batch)
+ * bytes, 16-byte aligned; lt_dqueue_init (re)initialises it on `stream`.
+ * lt_dqueue_push: ratio is device fp32 [batch, hq] (e.g. the ratio output of
+ * lt_prefill_attn_ratio for this layer).  A push that is invalid for a
+ * sequence (layer out of range or pushed twice, non-finite score) leaves that
+ * sequence's queue unchanged and sets an error bit that lt_dqueue_error
+ * reads (synchronously).  L, batch must match the values given to init.
+ * lt_dqueue_result writes lazy_mask (device uint8 [batch, L]) and, if not
+ * null, order (device int32 [batch, budget]: demoted layers in demotion
+ * order, -1 past the number demoted so far).
+ */
+size_t lt_dqueue_state_bytes(int L, int batch);
+lt_status lt_dqueue_init(void* state, int L, int budget, int batch, lt_stream stream);
+lt_status lt_dqueue_push(void* state, int L, int batch, int layer, const float* ratio, int hq, lt_stream stream);
+lt_status lt_dqueue_result(const void* state, int L, int batch, int budget, uint8_t* lazy_mask, int32_t* order,
+                           lt_stream stream);
+lt_status lt_dqueue_error(const void* state, int* error_bits);
+
+/*
+ * Compaction driven by the device queue: for every sequence b whose latest
+ * lt_dqueue_push demoted a layer m (the k-th demotion of b, k from 0), the
+ * streaming rows of layer m (as lt_compact_kv: p = [0, min(S,N)) ++
+ * [max(S, N-W), N), zero past the kept count) are written to pool slot k:
+ *   K_pool[k, b, kh, r, :] = K_m[cu[b] + p_r, kh, :],  pool_len[k, b] = |p|.
+ * Sequences with no demotion in the latest push are not touched.
+ * K_layers, V_layers: device arrays of L device pointers (layer l's K/V
+ * [T, hkv, d] bf16).  K_pool, V_pool: device bf16 [budget, batch, hkv, S+W, d];
+ * pool_len: device int32 [budget, batch].  Enqueue it right after the push
+ * (same stream) and before the next push.
+ */
+lt_status lt_compact_kv_pending(const lt_shape* shape, const void* const* K_layers, const void* const* V_layers,
+                                const void* state, int L, int budget, int S, int W, void* K_pool, void* V_pool,
+                                int32_t* pool_len, lt_stream stream);
+
+/*
+ * Decode on a demoted layer's streaming KV cache (press-release page: the
+ * converted layers use streaming attention with a constant-size KV cache).
+ * The cache is the [batch, hkv, S+W, d] bf16 layout lt_compact_kv writes, with
+ * stream_len[b] valid rows: rows [0, S) hold the sink positions and rows
+ * [S, S+W) the recent window, used as a ring once full.
+ *
+ * lt_stream_ring_init: next_slot[b] = stream_len[b] < S+W ? stream_len[b] : S,
+ * the slot the next token goes to (device int32 [batch]).  Call once after
+ * compaction.
+ * lt_stream_append: writes the new token's key and value (k_new, v_new: device
+ * bf16 [batch, hkv, d]) into slot next_slot[b] of every KV head, then advances
+ * stream_len / next_slot: while the cache is not full the token is appended;
+ * once full it replaces the window's oldest row.  The cache then holds the key
+ * set K_p = [0, min(S, p+1)) U [max(S, p-W+1), p] of the token at position p.
+ * W >= 1.  A sequence whose (stream_len, next_slot) no init/append sequence can
+ * produce (next_slot outside [0, S+W), or a non-full cache whose next_slot is
+ * not stream_len) is skipped: nothing is written for it.
+ * lt_stream_decode: for each sequence b and query head h (KV head h / g):
+ *   LSE[b, h] = log sum_{r < len} exp(scale q . K_s[b, kh, r]),
+ *   O[b, h]   = sum_r exp(scale q . K_s[b, kh, r] - LSE) V_s[b, kh, r]
+ * q, O: device bf16 [batch, hq, d]; LSE: device fp32 [batch, hq] (natural log;
+ * -inf and O = 0 for a sequence with no rows).  slots = S + W of the cache;
+ * stream_len[b] above slots is read as slots.  Errors: LT_ERR_INVALID_ARG for
+ * misaligned pointers (q, K/V, O 16 bytes), batch outside [1, 65535], hq not a
+ * multiple of hkv, slots < 1 or a non-finite scale; LT_ERR_UNSUPPORTED for
+ * head_dim other than 64 and 128.  Buffers are the caller's; nothing is
+ * allocated.  Asynchronous on `stream`.
+ */
+lt_status lt_stream_ring_init(const int32_t* stream_len, int32_t* next_slot, int batch, int S, int W,
+                              lt_stream stream);
+lt_status lt_stream_append(void* K_stream, void* V_stream, int32_t* stream_len, int32_t* next_slot, const void* k_new,
+                           const void* v_new, int batch, int hkv, int head_dim, int S, int W, lt_stream stream);
+lt_status lt_stream_decode(const void* q, const void* K_stream, const void* V_stream, const int32_t* stream_len,
+                           int batch, int hq, int hkv, int head_dim, int slots, void* O, float* LSE,
+                           float softmax_scale, lt_stream stream);
 
 /*
  * Device status word of the current device: LT_OK, or LT_ERR_TIMEOUT if a kernel

@@ -34,5 +34,16 @@ from .binding import (  # noqa: F401
     lt_status_string,
     lt_version,
     LayerQueue,
+    DeviceQueue,
+    layer_pointer_table,
+    lt_compact_kv_pending,
+    lt_dqueue_error,
+    lt_dqueue_init,
+    lt_dqueue_push,
+    lt_dqueue_result,
+    lt_dqueue_state_bytes,
+    lt_stream_append,
+    lt_stream_decode,
+    lt_stream_ring_init,
 )
 from .build import build  # noqa: F401

@@ -55,6 +55,15 @@ _SIGS = {
     "lt_queue_size": (_i, [_vp]),
     "lt_queue_destroy": (None, [_vp]),
     "lt_compact_kv": (_i, [_shp, _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _vp]),
+    "lt_dqueue_state_bytes": (ctypes.c_size_t, [_i, _i]),
+    "lt_dqueue_init": (_i, [_vp, _i, _i, _i, _vp]),
+    "lt_dqueue_push": (_i, [_vp, _i, _i, _i, _vp, _i, _vp]),
+    "lt_dqueue_result": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
+    "lt_dqueue_error": (_i, [_vp, ctypes.POINTER(_i)]),
+    "lt_compact_kv_pending": (_i, [_shp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "lt_stream_ring_init": (_i, [_vp, _vp, _i, _i, _i, _vp]),
+    "lt_stream_append": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
+    "lt_stream_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp]),
     "lt_device_status": (_i, [_i]),
     "lt_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "lt_status_string": (ctypes.c_char_p, [_i]),
@@ -320,3 +329,136 @@ def lt_device_status(clear: bool = True) -> int:
 def lt_selftest_wait_timeout(limit_us, stream=None):
     """Run the bounded-wait self-test kernel (see include/lt.h)."""
     _check(library().lt_selftest_wait_timeout(int(limit_us), _stream_handle(stream)), "lt_selftest_wait_timeout")
+
+
+def lt_dqueue_state_bytes(L, batch) -> int:
+    return int(library().lt_dqueue_state_bytes(int(L), int(batch)))
+
+
+def lt_dqueue_init(state, L, budget, batch, stream=None):
+    _dev_tensor(state, "state", torch.uint8, 1)
+    if state.numel() < lt_dqueue_state_bytes(L, batch):
+        raise ValueError("state is smaller than lt_dqueue_state_bytes(L, batch)")
+    _check(library().lt_dqueue_init(state.data_ptr(), int(L), int(budget), int(batch), _stream_handle(stream)),
+           "lt_dqueue_init")
+
+
+def lt_dqueue_push(state, L, batch, layer, ratio, stream=None):
+    _dev_tensor(state, "state", torch.uint8, 1)
+    _dev_tensor(ratio, "ratio", torch.float32, 2)
+    if ratio.shape[0] != batch:
+        raise ValueError("ratio must be [batch, hq]")
+    _check(library().lt_dqueue_push(state.data_ptr(), int(L), int(batch), int(layer), ratio.data_ptr(),
+                                    int(ratio.shape[1]), _stream_handle(stream)), "lt_dqueue_push")
+
+
+def lt_dqueue_result(state, L, batch, budget, lazy_mask=None, order=None, stream=None):
+    _dev_tensor(state, "state", torch.uint8, 1)
+    if lazy_mask is None:
+        lazy_mask = torch.empty((batch, L), dtype=torch.uint8, device=state.device)
+    if order is None:
+        order = torch.empty((batch, max(int(budget), 1)), dtype=torch.int32, device=state.device)
+    _check(library().lt_dqueue_result(state.data_ptr(), int(L), int(batch), int(budget), lazy_mask.data_ptr(),
+                                      order.data_ptr(), _stream_handle(stream)), "lt_dqueue_result")
+    return lazy_mask, order[:, : int(budget)]
+
+
+def lt_dqueue_error(state) -> int:
+    bits = ctypes.c_int(0)
+    _check(library().lt_dqueue_error(state.data_ptr(), ctypes.byref(bits)), "lt_dqueue_error")
+    return bits.value
+
+
+class DeviceQueue:
+    """Owning wrapper of one device-resident queue state for `batch` sequences."""
+
+    def __init__(self, L, budget, batch, device="cuda", stream=None):
+        self.L, self.budget, self.batch = int(L), int(budget), int(batch)
+        self.state = torch.empty(lt_dqueue_state_bytes(L, batch), dtype=torch.uint8, device=device)
+        lt_dqueue_init(self.state, L, budget, batch, stream)
+
+    def reset(self, stream=None):
+        lt_dqueue_init(self.state, self.L, self.budget, self.batch, stream)
+
+    def push(self, layer, ratio, stream=None):
+        lt_dqueue_push(self.state, self.L, self.batch, layer, ratio, stream)
+
+    def result(self, stream=None):
+        return lt_dqueue_result(self.state, self.L, self.batch, self.budget, stream=stream)
+
+    def error(self) -> int:
+        return lt_dqueue_error(self.state)
+
+
+def layer_pointer_table(tensors, device="cuda"):
+    """Device int64 array of the tensors' data pointers (for lt_compact_kv_pending)."""
+    return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64, device=device)
+
+
+def lt_compact_kv_pending(K_layers, V_layers, queue, S, W, K_pool, V_pool, pool_len, total_tokens, hkv, d,
+                          cu_seqlens=None, max_seqlen=None, stream=None):
+    """Compaction of the layers the latest device-queue push demoted (see include/lt.h).
+    K_layers / V_layers: device int64 pointer tables from layer_pointer_table."""
+    for t, n in ((K_layers, "K_layers"), (V_layers, "V_layers")):
+        _dev_tensor(t, n, torch.int64, 1)
+        if t.numel() != queue.L:
+            raise ValueError(f"{n} must hold L pointers")
+    slots = int(S) + int(W)
+    for t, n in ((K_pool, "K_pool"), (V_pool, "V_pool")):
+        _dev_tensor(t, n, torch.bfloat16, 5)
+        if t.shape != (queue.budget, queue.batch, hkv, slots, d):
+            raise ValueError(f"{n} must be [budget, batch, hkv, S+W, d]")
+    _dev_tensor(pool_len, "pool_len", torch.int32, 2)
+    shape = _shape(total_tokens, hkv, hkv, d, cu_seqlens, max_seqlen)
+    if shape.batch != queue.batch:
+        raise ValueError("batch differs from the queue's")
+    _check(library().lt_compact_kv_pending(ctypes.byref(shape), K_layers.data_ptr(), V_layers.data_ptr(),
+                                           queue.state.data_ptr(), queue.L, queue.budget, int(S), int(W),
+                                           K_pool.data_ptr(), V_pool.data_ptr(), pool_len.data_ptr(),
+                                           _stream_handle(stream)), "lt_compact_kv_pending")
+
+
+def lt_stream_ring_init(stream_len, next_slot, S, W, stream=None):
+    _dev_tensor(stream_len, "stream_len", torch.int32, 1)
+    _dev_tensor(next_slot, "next_slot", torch.int32, 1)
+    _check(library().lt_stream_ring_init(stream_len.data_ptr(), next_slot.data_ptr(), stream_len.numel(), int(S),
+                                         int(W), _stream_handle(stream)), "lt_stream_ring_init")
+
+
+def lt_stream_append(K_stream, V_stream, stream_len, next_slot, k_new, v_new, S, W, stream=None):
+    """Append one token per sequence (k_new, v_new [batch, hkv, d]) to the streaming cache."""
+    for t, n in ((K_stream, "K_stream"), (V_stream, "V_stream")):
+        _dev_tensor(t, n, torch.bfloat16, 4)
+    B, hkv, slots, d = K_stream.shape
+    if slots != S + W or V_stream.shape != K_stream.shape:
+        raise ValueError("caches must be [batch, hkv, S+W, d]")
+    for t, n in ((k_new, "k_new"), (v_new, "v_new")):
+        _dev_tensor(t, n, torch.bfloat16, 3)
+        if t.shape != (B, hkv, d):
+            raise ValueError(f"{n} must be [batch, hkv, d]")
+    _dev_tensor(stream_len, "stream_len", torch.int32, 1)
+    _dev_tensor(next_slot, "next_slot", torch.int32, 1)
+    _check(library().lt_stream_append(K_stream.data_ptr(), V_stream.data_ptr(), stream_len.data_ptr(),
+                                      next_slot.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), B, hkv, d, int(S),
+                                      int(W), _stream_handle(stream)), "lt_stream_append")
+
+
+def lt_stream_decode(q, K_stream, V_stream, stream_len, softmax_scale=None, out=None, lse=None, stream=None):
+    """Decode attention over the streaming cache: q [batch, hq, d] -> (O [batch, hq, d], LSE [batch, hq])."""
+    _dev_tensor(q, "q", torch.bfloat16, 3)
+    for t, n in ((K_stream, "K_stream"), (V_stream, "V_stream")):
+        _dev_tensor(t, n, torch.bfloat16, 4)
+    B, hq, d = q.shape
+    _, hkv, slots, dk = K_stream.shape
+    if K_stream.shape[0] != B or dk != d or V_stream.shape != K_stream.shape:
+        raise ValueError("caches must be [batch, hkv, S+W, d] with q's batch and d")
+    _dev_tensor(stream_len, "stream_len", torch.int32, 1)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    _check(library().lt_stream_decode(q.data_ptr(), K_stream.data_ptr(), V_stream.data_ptr(), stream_len.data_ptr(),
+                                      B, hq, hkv, d, slots, out.data_ptr(), lse.data_ptr(),
+                                      0.0 if softmax_scale is None else float(softmax_scale), _stream_handle(stream)),
+           "lt_stream_decode")
+    return out, lse

@@ -13,8 +13,10 @@
 
 #include "attn_fwd.cuh"
 #include "compact_kv.cuh"
+#include "dqueue.cuh"
 #include "lazy_ratio.cuh"
 #include "selftest.cuh"
+#include "stream_decode.cuh"
 #include "lt.h"
 
 namespace {
@@ -283,6 +285,147 @@ lt_status lt_compact_kv(const lt_shape* shape, const void* K, const void* V, con
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   lt::compact_kv_kernel<<<int(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+size_t lt_dqueue_state_bytes(int L, int batch) {
+  if (L < 1 || batch < 1) return 0;
+  return lt::dqueue_bytes(L, batch);
+}
+
+static bool dq_args(const void* state, int L, int batch) {
+  return aligned(state, 16) && L >= 1 && L <= 4096 && batch >= 1 && batch <= (1 << 20);
+}
+
+static int dq_blocks(int batch) { return (batch + 127) / 128; }
+
+lt_status lt_dqueue_init(void* state, int L, int budget, int batch, lt_stream stream) {
+  if (!dq_args(state, L, batch) || budget < 0 || budget > L) return LT_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  lt_status st = device_info(&dev);
+  if (st != LT_OK) return st;
+  lt::dqueue_init_kernel<<<dq_blocks(batch), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(state, L, budget,
+                                                                                               batch);
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_dqueue_push(void* state, int L, int batch, int layer, const float* ratio, int hq, lt_stream stream) {
+  if (!dq_args(state, L, batch) || !aligned(ratio, 4) || hq < 1) return LT_ERR_INVALID_ARG;
+  lt::dqueue_push_kernel<<<dq_blocks(batch), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(state, L, batch,
+                                                                                               layer, ratio, hq);
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_dqueue_result(const void* state, int L, int batch, int budget, uint8_t* lazy_mask, int32_t* order,
+                           lt_stream stream) {
+  if (!dq_args(state, L, batch) || !lazy_mask || budget < 0 || budget > L || (order && !aligned(order, 4)))
+    return LT_ERR_INVALID_ARG;
+  lt::dqueue_result_kernel<<<dq_blocks(batch), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      state, L, batch, budget, lazy_mask, order);
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_dqueue_error(const void* state, int* error_bits) {
+  if (!aligned(state, 16) || !error_bits) return LT_ERR_INVALID_ARG;
+  int32_t w = 0;
+  if (cudaMemcpy(&w, static_cast<const int32_t*>(state) + 3, sizeof w, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return LT_ERR_CUDA;
+  *error_bits = w;
+  return LT_OK;
+}
+
+lt_status lt_compact_kv_pending(const lt_shape* shape, const void* const* K_layers, const void* const* V_layers,
+                                const void* state, int L, int budget, int S, int W, void* K_pool, void* V_pool,
+                                int32_t* pool_len, lt_stream stream) {
+  lt_status st = check_shape(shape);
+  if (st != LT_OK) return st;
+  if (!aligned(K_layers, 8) || !aligned(V_layers, 8) || !dq_args(state, L, shape->batch) || budget < 1 ||
+      budget > L || !aligned(K_pool, 16) || !aligned(V_pool, 16) || !aligned(pool_len, 4))
+    return LT_ERR_INVALID_ARG;
+  if (S < 0 || W < 0 || (long long)S + W < 1 || (long long)S + W > (1 << 24)) return LT_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != LT_OK) return st;
+  lt::CompactPendingParams p;
+  p.batch = shape->batch;
+  p.total_tokens = shape->total_tokens;
+  p.hkv = shape->hkv;
+  p.D = shape->head_dim;
+  p.S = S;
+  p.W = W;
+  p.L = L;
+  p.budget = budget;
+  p.cu_seqlens = shape->cu_seqlens;
+  p.K_layers = reinterpret_cast<const uint4* const*>(K_layers);
+  p.V_layers = reinterpret_cast<const uint4* const*>(V_layers);
+  p.state = state;
+  p.K_pool = static_cast<uint4*>(K_pool);
+  p.V_pool = static_cast<uint4*>(V_pool);
+  p.pool_len = pool_len;
+  const long long work = (long long)shape->batch * (S + W) * shape->hkv * (shape->head_dim / 8);
+  long long blocks = (work + 255) / 256;
+  const long long cap = (long long)dev->sm_count * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  lt::compact_pending_kernel<<<int(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_stream_ring_init(const int32_t* stream_len, int32_t* next_slot, int batch, int S, int W,
+                              lt_stream stream) {
+  if (!aligned(stream_len, 4) || !aligned(next_slot, 4) || batch < 1 || S < 0 || W < 1) return LT_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  lt_status st = device_info(&dev);
+  if (st != LT_OK) return st;
+  lt::stream_ring_init_kernel<<<(batch + 127) / 128, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      stream_len, next_slot, batch, S, W);
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_stream_append(void* K_stream, void* V_stream, int32_t* stream_len, int32_t* next_slot, const void* k_new,
+                           const void* v_new, int batch, int hkv, int head_dim, int S, int W, lt_stream stream) {
+  if (!aligned(K_stream, 16) || !aligned(V_stream, 16) || !aligned(stream_len, 4) || !aligned(next_slot, 4) ||
+      !aligned(k_new, 16) || !aligned(v_new, 16) || batch < 1 || hkv < 1 || S < 0 || W < 1)
+    return LT_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return LT_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  lt_status st = device_info(&dev);
+  if (st != LT_OK) return st;
+  lt::stream_append_kernel<<<batch, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(K_stream), static_cast<uint4*>(V_stream), stream_len, next_slot,
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), hkv, head_dim, S, W);
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_stream_decode(const void* q, const void* K_stream, const void* V_stream, const int32_t* stream_len,
+                           int batch, int hq, int hkv, int head_dim, int slots, void* O, float* LSE,
+                           float softmax_scale, lt_stream stream) {
+  if (!aligned(q, 16) || !aligned(K_stream, 16) || !aligned(V_stream, 16) || !aligned(stream_len, 4) ||
+      !aligned(O, 16) || !aligned(LSE, 4) || batch < 1 || batch > 65535 || hq < 1 || hkv < 1 || hq % hkv ||
+      slots < 1 || !std::isfinite(softmax_scale))
+    return LT_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return LT_ERR_UNSUPPORTED;
+  DeviceInfo* dev = nullptr;
+  lt_status st = device_info(&dev);
+  if (st != LT_OK) return st;
+  lt::DecodeParams p;
+  p.batch = batch;
+  p.hq = hq;
+  p.hkv = hkv;
+  p.group = hq / hkv;
+  p.slots = slots;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.K = static_cast<const __nv_bfloat16*>(K_stream);
+  p.V = static_cast<const __nv_bfloat16*>(V_stream);
+  p.len = stream_len;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.LSE = LSE;
+  p.scale_log2 = resolve_scale(softmax_scale, head_dim) * kLog2e;
+  const dim3 grid(hkv, batch);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (head_dim == 64)
+    lt::stream_decode_kernel<64><<<grid, 128, 0, s>>>(p);
+  else
+    lt::stream_decode_kernel<128><<<grid, 128, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
 }
 

@@ -58,6 +58,8 @@ def _configure(lib):
                                         ctypes.POINTER(ctypes.c_int)]
     lib.oracle_compact_kv.argtypes = [_i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _u16p, _u16p, _u8p,
                                       ctypes.c_int, ctypes.c_int, _u16p, _u16p, _i32p]
+    lib.oracle_attn_keys.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _u16p, _u16p, _u16p, _i32p,
+                                     ctypes.c_double, _f64p, _f64p]
     return lib
 
 
@@ -232,3 +234,23 @@ def compact_kv(cu_seqlens, K, V, mask, S, W, Ks=None, Vs=None):
                                  int(S), int(W), _ptr(Ks, _u16p), _ptr(Vs, _u16p), _ptr(ln, _i32p)):
         raise ValueError("oracle_compact_kv failed")
     return Ks, Vs, ln
+
+
+def attn_keys(q, K, V, m, scale=None):
+    """Attention of each query row over its own key rows (decode over a
+    streaming cache).  q [n, d], K/V [n, m_max, d] uint16 bf16 bits, m [n] keys
+    used per item.  Returns (O [n, d] float64, LSE [n] float64)."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    K = np.ascontiguousarray(K, dtype=np.uint16)
+    V = np.ascontiguousarray(V, dtype=np.uint16)
+    m = np.ascontiguousarray(m, dtype=np.int32)
+    n, d = q.shape
+    if K.shape != V.shape or K.shape[0] != n or K.shape[2] != d or m.shape != (n,):
+        raise ValueError("q [n, d], K/V [n, m_max, d], m [n]")
+    O = np.empty((n, d), np.float64)
+    LSE = np.empty((n,), np.float64)
+    rc = _load().oracle_attn_keys(n, K.shape[1], d, _ptr(q, _u16p), _ptr(K, _u16p), _ptr(V, _u16p), _ptr(m, _i32p),
+                                  default_scale(d) if scale is None else float(scale), _ptr(O, _f64p), _ptr(LSE, _f64p))
+    if rc:
+        raise ValueError(f"oracle_attn_keys failed ({rc})")
+    return O, LSE

@@ -48,6 +48,12 @@
  *  - oracle_compact_kv: the streaming version of a demoted layer's KV cache keeps
  *    the rows p = [0, min(S, N)) ++ [max(S, N - W), N) of every KV head.
  *
+ *  - oracle_attn_keys: attention of one query row over an explicit set of key
+ *    rows -- what a streaming (sink + recent window) layer computes at decode
+ *    (press-release page: the converted layers use streaming attention, which
+ *    needs only a constant-size KV cache):
+ *        LSE = log sum_j exp(scale q.k_j),  O = sum_j exp(scale q.k_j - LSE) v_j.
+ *
  * Inputs are bf16 bit patterns (uint16), decoded exactly to double.  All
  * arithmetic is fp64 with libm exp/log.
  */
@@ -467,5 +473,46 @@ int oracle_compact_kv(const int32_t* cu_seqlens, int batch, int hkv, int d, cons
       }
     len[b] = n;
   }
+  return 0;
+}
+
+/* ------------------------------------------------------- keyed attention */
+
+/*
+ * Item n: query q[n, :] against the first m[n] rows of K[n, :, :], V[n, :, :]
+ * (each [m_max, d], bf16 bits).  O: [n_items, d]; LSE: [n_items].  An item with
+ * no keys gets O = 0 and LSE = -inf.
+ */
+int oracle_attn_keys(int64_t n_items, int m_max, int d, const uint16_t* q, const uint16_t* K, const uint16_t* V,
+                     const int32_t* m, double scale, double* O, double* LSE) {
+  if (n_items < 0 || m_max < 0 || d < 1 || (n_items > 0 && (!q || !K || !V || !m || !O || !LSE))) return -1;
+  double* s = (double*)malloc(sizeof(double) * (size_t)(m_max > 0 ? m_max : 1));
+  if (!s) return -2;
+  for (int64_t it = 0; it < n_items; ++it) {
+    const int mk = m[it];
+    if (mk < 0 || mk > m_max) { free(s); return -1; }
+    const uint16_t* qr = q + (size_t)it * d;
+    double* o = O + (size_t)it * d;
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    if (mk == 0) { LSE[it] = -INFINITY; continue; }
+    double mx = -INFINITY;
+    for (int j = 0; j < mk; ++j) {
+      const uint16_t* kr = K + ((size_t)it * m_max + j) * d;
+      double acc = 0.0;
+      for (int c = 0; c < d; ++c) acc += bf16_bits_to_double(qr[c]) * bf16_bits_to_double(kr[c]);
+      s[j] = scale * acc;
+      if (s[j] > mx) mx = s[j];
+    }
+    double sum = 0.0;
+    for (int j = 0; j < mk; ++j) sum += exp(s[j] - mx);
+    const double lse = mx + log(sum);
+    for (int j = 0; j < mk; ++j) {
+      const double w = exp(s[j] - lse);
+      const uint16_t* vr = V + ((size_t)it * m_max + j) * d;
+      for (int c = 0; c < d; ++c) o[c] += w * bf16_bits_to_double(vr[c]);
+    }
+    LSE[it] = lse;
+  }
+  free(s);
   return 0;
 }

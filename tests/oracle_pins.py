@@ -405,4 +405,49 @@ def pin_compaction_matches_slicing():
         assert np.all(Ks[b][:, len(keep):] == 0) and np.all(Vs[b][:, len(keep):] == 0)
 
 
+# ------------------------------------------------------ keyed-attention pins
+
+def pin_keyed_attention_matches_scipy():
+    rng = np.random.default_rng(51)
+    n, m_max, d = 6, 9, 8
+    q = rand_bf16(rng, (n, d), 1.5)
+    K, V = rand_bf16(rng, (n, m_max, d), 1.5), rand_bf16(rng, (n, m_max, d))
+    m = np.array([9, 1, 4, 0, 7, 9], np.int32)
+    O, LSE = oracle.attn_keys(q, K, V, m, scale=0.4)
+    for i in range(n):
+        if m[i] == 0:
+            assert LSE[i] == -np.inf and np.all(O[i] == 0)
+            continue
+        row = 0.4 * values_of(K[i, : m[i]]) @ values_of(q[i])
+        assert abs(LSE[i] - logsumexp(row)) < 1e-12
+        assert np.allclose(O[i], softmax(row) @ values_of(V[i, : m[i]]), atol=1e-12)
+
+
+def pin_keyed_attention_uniform():
+    rng = np.random.default_rng(52)
+    K, V = rand_bf16(rng, (2, 5, 4)), rand_bf16(rng, (2, 5, 4))
+    O, LSE = oracle.attn_keys(np.zeros((2, 4), np.uint16), K, V, np.array([5, 3], np.int32))
+    assert np.allclose(LSE, np.log([5, 3]), atol=1e-15)
+    assert np.allclose(O[1], values_of(V[1, :3]).mean(axis=0), atol=1e-15)
+
+
+def pin_streaming_normaliser_is_lse_plus_log_ratio():
+    """Over the key set K_i of row i, log sum exp(s_ij) = LSE_i + log r_i: the
+    streaming attention's normaliser is the full one times the lazy ratio."""
+    cu, Q, K = _ratio_problem(53, lengths=(37, 12), hq=2, hkv=1, d=8)
+    V = rand_bf16(np.random.default_rng(54), K.shape)
+    S, W = 3, 5
+    _, LSE = oracle.attn(cu, Q, K, V)
+    for b in range(len(cu) - 1):
+        t = int(cu[b + 1] - 1)
+        i = int(t - cu[b])
+        keys = sorted(key_set(i, S, W))
+        for h in range(Q.shape[1]):
+            r = oracle.lazy_ratio_rows(cu, Q, K, S, W, np.array([t]), np.array([h]))[0]
+            Ks = np.ascontiguousarray(K[[cu[b] + j for j in keys], 0][None])
+            Vs = np.ascontiguousarray(V[[cu[b] + j for j in keys], 0][None])
+            _, lse_s = oracle.attn_keys(np.ascontiguousarray(Q[t, h][None]), Ks, Vs, np.array([len(keys)], np.int32))
+            assert abs(lse_s[0] - (LSE[h, t] + np.log(r))) < 1e-12
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

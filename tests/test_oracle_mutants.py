@@ -33,6 +33,9 @@ MUTANTS = [
     ("compaction window one short", "const int recent = pos >= N - W && pos >= S;", "const int recent = pos > N - W && pos >= S;"),
     ("compaction keeps no sinks", "const int sink = pos < S;", "const int sink = 0;"),
     ("compaction tail not zeroed", "memset(Ks + dst, 0, sizeof(uint16_t) * (size_t)d);", ";"),
+    ("keyed attention drops scale", "s[j] = scale * acc;", "s[j] = acc;"),
+    ("keyed attention skips last key", "for (int j = 0; j < mk; ++j) sum += exp(s[j] - mx);", "for (int j = 0; j + 1 < mk; ++j) sum += exp(s[j] - mx);"),
+    ("keyed attention wrong value row", "const uint16_t* vr = V + ((size_t)it * m_max + j) * d;", "const uint16_t* vr = V + ((size_t)it * m_max) * d;"),
 ]
 
 
