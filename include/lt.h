@@ -254,6 +254,18 @@ lt_status lt_compact_kv_pending(const lt_shape* shape, const void* const* K_laye
  * multiple of hkv, slots < 1 or a non-finite scale; LT_ERR_UNSUPPORTED for
  * head_dim other than 64 and 128.  Buffers are the caller's; nothing is
  * allocated.  Asynchronous on `stream`.
+ *
+ * lt_decode_attn: the same decode step on a kept (full-attention) layer's
+ * cache, token-major K/V [rows, hkv, d] bf16 with the rows of one sequence
+ * contiguous: sequence b's position r is row seq_start[b] + r (device int32
+ * [batch], e.g. the prefill's cu_seqlens) or, with seq_start NULL, row
+ * b * seq_capacity + r (a padded [batch, seq_capacity, hkv, d] cache).  len:
+ * device int32 [batch], positions attended (read clamped to [0, max_len]);
+ * max_len >= 1 bounds every len[b] (and seq_capacity >= max_len when seq_start
+ * is NULL).  The caller guarantees the rows read lie inside K and V.  O and LSE
+ * as for lt_stream_decode.  Both decode calls split each (sequence, KV head)
+ * over a cluster of up to 16 CTAs merged in distributed shared memory; no
+ * memory beyond the arguments is written.
  */
 lt_status lt_stream_ring_init(const int32_t* stream_len, int32_t* next_slot, int batch, int S, int W,
                               lt_stream stream);
@@ -262,6 +274,9 @@ lt_status lt_stream_append(void* K_stream, void* V_stream, int32_t* stream_len, 
 lt_status lt_stream_decode(const void* q, const void* K_stream, const void* V_stream, const int32_t* stream_len,
                            int batch, int hq, int hkv, int head_dim, int slots, void* O, float* LSE,
                            float softmax_scale, lt_stream stream);
+lt_status lt_decode_attn(const void* q, const void* K, const void* V, const int32_t* seq_start, int seq_capacity,
+                         const int32_t* len, int batch, int hq, int hkv, int head_dim, int max_len, void* O,
+                         float* LSE, float softmax_scale, lt_stream stream);
 
 /*
  * Device status word of the current device: LT_OK, or LT_ERR_TIMEOUT if a kernel

@@ -44,6 +44,7 @@ from .binding import (  # noqa: F401
     lt_dqueue_state_bytes,
     lt_stream_append,
     lt_stream_decode,
+    lt_decode_attn,
     lt_stream_ring_init,
 )
 from .build import build  # noqa: F401

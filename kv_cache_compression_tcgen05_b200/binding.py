@@ -64,6 +64,7 @@ _SIGS = {
     "lt_stream_ring_init": (_i, [_vp, _vp, _i, _i, _i, _vp]),
     "lt_stream_append": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "lt_stream_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp]),
+    "lt_decode_attn": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp]),
     "lt_device_status": (_i, [_i]),
     "lt_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "lt_status_string": (ctypes.c_char_p, [_i]),
@@ -461,4 +462,46 @@ def lt_stream_decode(q, K_stream, V_stream, stream_len, softmax_scale=None, out=
                                       B, hq, hkv, d, slots, out.data_ptr(), lse.data_ptr(),
                                       0.0 if softmax_scale is None else float(softmax_scale), _stream_handle(stream)),
            "lt_stream_decode")
+    return out, lse
+
+
+def lt_decode_attn(q, K, V, seq_len, seq_start=None, max_len=None, softmax_scale=None, out=None, lse=None,
+                   stream=None):
+    """Decode attention over a kept layer's full cache: q [batch, hq, d] ->
+    (O [batch, hq, d], LSE [batch, hq]).  K/V either token-major packed
+    [rows, hkv, d] with seq_start (device int32 [batch], first row of each
+    sequence), or padded [batch, capacity, hkv, d] with seq_start None.
+    seq_len: device int32 [batch] positions attended."""
+    _dev_tensor(q, "q", torch.bfloat16, 3)
+    B, hq, d = q.shape
+    if K.dim() == 4:
+        for t, n in ((K, "K"), (V, "V")):
+            _dev_tensor(t, n, torch.bfloat16, 4)
+        if seq_start is not None:
+            raise ValueError("a padded [batch, capacity, hkv, d] cache takes no seq_start")
+        Bk, cap, hkv, dk = K.shape
+        if Bk != B:
+            raise ValueError("padded cache batch differs from q's")
+        limit = cap if max_len is None else int(max_len)
+    else:
+        for t, n in ((K, "K"), (V, "V")):
+            _dev_tensor(t, n, torch.bfloat16, 3)
+        if seq_start is None:
+            raise ValueError("a packed [rows, hkv, d] cache needs seq_start")
+        _dev_tensor(seq_start, "seq_start", torch.int32, 1)
+        rows, hkv, dk = K.shape
+        cap = 0
+        limit = rows if max_len is None else int(max_len)
+    if dk != d or V.shape != K.shape:
+        raise ValueError("K and V must have the same shape and q's head dim")
+    _dev_tensor(seq_len, "seq_len", torch.int32, 1)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    _check(library().lt_decode_attn(q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                    None if seq_start is None else seq_start.data_ptr(), cap, seq_len.data_ptr(), B,
+                                    hq, hkv, d, limit, out.data_ptr(), lse.data_ptr(),
+                                    0.0 if softmax_scale is None else float(softmax_scale), _stream_handle(stream)),
+           "lt_decode_attn")
     return out, lse

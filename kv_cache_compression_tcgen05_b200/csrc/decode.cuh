@@ -1,0 +1,287 @@
+// decode.cuh -- one decode step of attention over a layer's KV cache: the
+// streaming cache of a demoted layer, or the full cache of a kept one.
+//
+// Press-release page ("LLM突破：推理加速，长CoT生成惊艳"): the converted layers
+// use streaming attention, which needs only a constant-size KV cache, while the
+// other layers keep full attention; the LightTransfer project page: the lazy
+// layers pay attention mostly to the initial and the recent tokens.  After
+// compaction a lazy layer keeps, per sequence and KV head, S + W rows: the S
+// sink positions and the W most recent ones.  At decode the new token's
+// key/value enter the window (replacing its oldest row once the cache is full)
+// and the token attends to the cached rows:
+//     K_p = [0, min(S, p+1)) U [max(S, p-W+1), p]   (p = the token's position)
+// -- the same key set the lazy ratio measures.  A kept layer's token attends
+// to all of its sequence's rows.
+//
+// Streaming cache layout: [batch, hkv, S+W, d] bf16 (as lt_compact_kv writes
+// it), len[b] valid rows; rows [0, S) are the sinks, rows [S, S+W) the window,
+// used as a ring once full: next[b] is the slot the next token goes to.
+// Full cache layout: token-major [rows, hkv, d] bf16, the rows of one sequence
+// contiguous (the prefill's packed K/V, or a padded [batch, capacity, hkv, d]).
+//
+// The decode is HBM bound: each cached row is read once per KV head for all g
+// query heads of its group, 4 per pass.  The rows of one (sequence, KV head)
+// are split over a cluster of `splits` CTAs; in a CTA each group of d/8 lanes
+// of a warp takes one row at a time, 8 elements per lane in one 16-byte load
+// (the next row's loads in flight while the current one is used), scores are
+// reduced over the group's lanes with shuffles, and each group keeps a running
+// (max, sum, output) per head in the log2 domain.  Groups merge through shuffles, warps through shared memory
+// and the cluster's CTAs through distributed shared memory into CTA rank 0,
+// which writes O and LSE.
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "lt_device.cuh"
+
+namespace lt {
+
+namespace dcg = cooperative_groups;
+
+__global__ void stream_ring_init_kernel(const int32_t* len, int32_t* next, int batch, int S, int W) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < batch) next[b] = len[b] < S + W ? len[b] : S;
+}
+
+// One CTA per sequence: the new rows of every KV head go to slot next[b]; then
+// one thread advances len and next.  len > S+W is read as a full cache.
+__global__ void stream_append_kernel(uint4* Ks, uint4* Vs, int32_t* len, int32_t* next, const uint4* k_new,
+                                     const uint4* v_new, int hkv, int D, int S, int W) {
+  const int b = blockIdx.x;
+  const int slots = S + W;
+  const int slot = next[b];
+  const int n = len[b];
+  // A state no ring operation can produce (slot outside the cache, or a free
+  // slot other than the one after the last row) is left untouched.
+  if (slot < 0 || slot >= slots || n < 0 || (n < slots && slot != n)) return;
+  const int pieces = D / 8;
+  for (int x = threadIdx.x; x < hkv * pieces; x += blockDim.x) {
+    const int kh = x / pieces, piece = x - kh * pieces;
+    const size_t dst = ((size_t(b) * hkv + kh) * slots + slot) * pieces + piece;
+    const size_t src = (size_t(b) * hkv + kh) * pieces + piece;
+    Ks[dst] = k_new[src];
+    Vs[dst] = v_new[src];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (n < slots) {
+      len[b] = n + 1;
+      next[b] = n + 1 < slots ? n + 1 : S;
+    } else {
+      next[b] = S + (slot - S + 1) % W;
+    }
+  }
+}
+
+// Element offsets: row r of KV head kh of sequence b starts at
+//   (seq_start ? seq_start[b] * row_stride : b * seq_stride) + r * row_stride + kh * head_stride.
+struct DecodeParams {
+  int batch, hq, hkv, group, splits, max_len;
+  const __nv_bfloat16* q;    // [batch, hq, d]
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  const int32_t* seq_start;  // [batch] first row of each sequence, or null
+  long long seq_stride, row_stride, head_stride;
+  const int32_t* len;        // [batch] valid rows (clamped to [0, max_len])
+  __nv_bfloat16* O;          // [batch, hq, d]
+  float* LSE;                // [batch, hq]
+  float scale_log2;
+};
+
+constexpr int kDecodeThreads = 256;
+constexpr int kDecodeWarps = kDecodeThreads / 32;
+constexpr int kDecodeHeads = 4;   // query heads per pass over the cache
+constexpr int kDecodeMaxSplits = 16;
+
+// Merges running softmax state (m2, l2, o2) into (m1, l1, o1); log2 domain.
+template <int E>
+__device__ __forceinline__ void softmax_merge(float& m1, float& l1, float (&o1)[E], float m2, float l2,
+                                              const float (&o2)[E]) {
+  const float M = fmaxf(m1, m2);
+  const float c1 = M == -INFINITY ? 0.f : fast_exp2(m1 - M);
+  const float c2 = M == -INFINITY ? 0.f : fast_exp2(m2 - M);
+  l1 = l1 * c1 + l2 * c2;
+#pragma unroll
+  for (int e = 0; e < E; ++e) o1[e] = o1[e] * c1 + o2[e] * c2;
+  m1 = M;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeParams p) {
+  constexpr int E = 8;           // elements of a row per lane (one 16-byte load)
+  constexpr int LPR = D / E;     // lanes per row
+  constexpr int GPW = 32 / LPR;  // row groups per warp
+  dcg::cluster_group cluster = dcg::this_cluster();
+  const int split = int(cluster.block_rank());
+  const int kh = blockIdx.x / p.splits;
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rgw = lane / LPR;  // row group in the warp
+  const int li = lane % LPR;   // lane in the row group
+  __shared__ float sm_m[kDecodeWarps][kDecodeHeads], sm_l[kDecodeWarps][kDecodeHeads];
+  __shared__ __align__(16) float sm_o[kDecodeWarps][kDecodeHeads][D];
+  __shared__ float cta_m[kDecodeHeads], cta_l[kDecodeHeads];
+  __shared__ __align__(16) float cta_o[kDecodeHeads][D];
+
+  const int n = min(max(p.len[b], 0), p.max_len);
+  const int chunk = (n + p.splits - 1) / p.splits;
+  const int r_begin = min(n, split * chunk);
+  const int r_end = min(n, r_begin + chunk);
+  const long long seq_off = p.seq_start ? (long long)p.seq_start[b] * p.row_stride : (long long)b * p.seq_stride;
+  const __nv_bfloat16* Kb = p.K + seq_off + kh * p.head_stride + li * E;
+  const __nv_bfloat16* Vb = p.V + seq_off + kh * p.head_stride + li * E;
+  constexpr int kRowsPerIter = kDecodeWarps * GPW;
+
+  for (int h0 = 0; h0 < p.group; h0 += kDecodeHeads) {
+    const int nh = min(kDecodeHeads, p.group - h0);
+    float q[kDecodeHeads][E];
+#pragma unroll
+    for (int hh = 0; hh < kDecodeHeads; ++hh) {
+      const int h = kh * p.group + h0 + min(hh, nh - 1);
+      const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(p.q + (size_t(b) * p.hq + h) * D + li * E));
+      const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        q[hh][2 * t] = __uint_as_float(w[t] << 16) * p.scale_log2;
+        q[hh][2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u) * p.scale_log2;
+      }
+    }
+    float m[kDecodeHeads], l[kDecodeHeads], o[kDecodeHeads][E];
+#pragma unroll
+    for (int hh = 0; hh < kDecodeHeads; ++hh) {
+      m[hh] = -INFINITY;
+      l[hh] = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[hh][e] = 0.f;
+    }
+    // Each warp takes GPW consecutive rows per iteration; the loop bound is
+    // warp-uniform so that every lane reaches every shuffle.
+    uint4 kc = make_uint4(0u, 0u, 0u, 0u), vc = kc;
+    {
+      const int row = r_begin + warp * GPW + rgw;
+      if (row < r_end) {
+        kc = __ldg(reinterpret_cast<const uint4*>(Kb + row * p.row_stride));
+        vc = __ldg(reinterpret_cast<const uint4*>(Vb + row * p.row_stride));
+      }
+    }
+    for (int rb = r_begin + warp * GPW; rb < r_end; rb += kRowsPerIter) {
+      const int row = rb + rgw;
+      const int row_next = row + kRowsPerIter;
+      uint4 kn = make_uint4(0u, 0u, 0u, 0u), vn = kn;
+      if (row_next < r_end) {
+        kn = __ldg(reinterpret_cast<const uint4*>(Kb + row_next * p.row_stride));
+        vn = __ldg(reinterpret_cast<const uint4*>(Vb + row_next * p.row_stride));
+      }
+      float k[E], v[E];
+      {
+        const uint32_t kw[4] = {kc.x, kc.y, kc.z, kc.w}, vw[4] = {vc.x, vc.y, vc.z, vc.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          k[2 * t] = __uint_as_float(kw[t] << 16);
+          k[2 * t + 1] = __uint_as_float(kw[t] & 0xFFFF0000u);
+          v[2 * t] = __uint_as_float(vw[t] << 16);
+          v[2 * t + 1] = __uint_as_float(vw[t] & 0xFFFF0000u);
+        }
+      }
+      const bool valid = row < r_end;
+#pragma unroll
+      for (int hh = 0; hh < kDecodeHeads; ++hh) {
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) s = fmaf(q[hh][e], k[e], s);
+#pragma unroll
+        for (int off = 1; off < LPR; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        if (valid) {
+          const float m_new = fmaxf(m[hh], s);
+          const float corr = fast_exp2(m[hh] - m_new);   // 0 on the group's first row (m = -inf)
+          const float w = fast_exp2(s - m_new);
+          l[hh] = l[hh] * corr + w;
+#pragma unroll
+          for (int e = 0; e < E; ++e) o[hh][e] = fmaf(o[hh][e], corr, w * v[e]);
+          m[hh] = m_new;
+        }
+      }
+      kc = kn;
+      vc = vn;
+    }
+    // Merge the GPW row groups of the warp (lanes li + LPR * g).
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+      for (int hh = 0; hh < kDecodeHeads; ++hh) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m[hh], off);
+        const float l2 = __shfl_xor_sync(0xffffffffu, l[hh], off);
+        float o2[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) o2[e] = __shfl_xor_sync(0xffffffffu, o[hh][e], off);
+        softmax_merge<E>(m[hh], l[hh], o[hh], m2, l2, o2);
+      }
+    }
+    if (rgw == 0) {
+#pragma unroll
+      for (int hh = 0; hh < kDecodeHeads; ++hh) {
+        if (li == 0) {
+          sm_m[warp][hh] = m[hh];
+          sm_l[warp][hh] = l[hh];
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) sm_o[warp][hh][li * E + e] = o[hh][e];
+      }
+    }
+    __syncthreads();
+    // Warp 0, row group 0: merge the warps into the CTA's partial state.
+    if (warp == 0 && rgw == 0) {
+#pragma unroll
+      for (int hh = 0; hh < kDecodeHeads; ++hh) {
+        float mm = sm_m[0][hh], ll = sm_l[0][hh], oo[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) oo[e] = sm_o[0][hh][li * E + e];
+        for (int w2 = 1; w2 < kDecodeWarps; ++w2) {
+          float o2[E];
+#pragma unroll
+          for (int e = 0; e < E; ++e) o2[e] = sm_o[w2][hh][li * E + e];
+          softmax_merge<E>(mm, ll, oo, sm_m[w2][hh], sm_l[w2][hh], o2);
+        }
+        if (li == 0) {
+          cta_m[hh] = mm;
+          cta_l[hh] = ll;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) cta_o[hh][li * E + e] = oo[e];
+      }
+    }
+    cluster.sync();   // every CTA's partial state is visible cluster-wide
+    // Rank 0, warp 0, row group 0: merge the cluster's CTAs in rank order and
+    // write the result.
+    if (split == 0 && warp == 0 && rgw == 0) {
+#pragma unroll
+      for (int hh = 0; hh < kDecodeHeads; ++hh) {
+        float mm = cta_m[hh], ll = cta_l[hh], oo[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) oo[e] = cta_o[hh][li * E + e];
+        for (int r = 1; r < p.splits; ++r) {
+          const float* rm = cluster.map_shared_rank(&cta_m[0], r);
+          const float* rl = cluster.map_shared_rank(&cta_l[0], r);
+          const float* ro = cluster.map_shared_rank(&cta_o[0][0], r);
+          float o2[E];
+#pragma unroll
+          for (int e = 0; e < E; ++e) o2[e] = ro[hh * D + li * E + e];
+          softmax_merge<E>(mm, ll, oo, rm[hh], rl[hh], o2);
+        }
+        if (hh < nh) {
+          const int h = kh * p.group + h0 + hh;
+          const float inv = ll > 0.f ? 1.f / ll : 0.f;
+          __nv_bfloat16* orow = p.O + (size_t(b) * p.hq + h) * D + li * E;
+#pragma unroll
+          for (int e = 0; e < E; e += 2)
+            *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(oo[e] * inv, oo[e + 1] * inv);
+          if (li == 0)
+            p.LSE[size_t(b) * p.hq + h] = ll > 0.f ? (mm + fast_log2(ll)) * 0.69314718055994531f : -INFINITY;
+        }
+      }
+    }
+    cluster.sync();   // rank 0 is done reading before any CTA's state is reused or released
+  }
+}
+
+}  // namespace lt

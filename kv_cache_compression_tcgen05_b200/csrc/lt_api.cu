@@ -16,7 +16,7 @@
 #include "dqueue.cuh"
 #include "lazy_ratio.cuh"
 #include "selftest.cuh"
-#include "stream_decode.cuh"
+#include "decode.cuh"
 #include "lt.h"
 
 namespace {
@@ -31,6 +31,7 @@ struct DeviceInfo {
   bool ready = false;
   int sm_count = 0;
   unsigned* status = nullptr;  // device address of g_status_word
+  int max_decode_splits = 8;   // largest cluster the decode kernels launch with
 };
 
 std::mutex g_mutex;
@@ -62,6 +63,30 @@ lt_status device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(lt::lazy_ratio_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              lt::RatioLayout<128>::bytes(lt::kRatioMaxGroup * 256)) != cudaSuccess)
       return LT_ERR_CUDA;
+    // Clusters of 16 CTAs are beyond the portable size: use them for the decode
+    // split only where the device reports that one fits.
+    info.max_decode_splits = 8;
+    if (cudaFuncSetAttribute(lt::decode_kernel<64>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess &&
+        cudaFuncSetAttribute(lt::decode_kernel<128>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess) {
+      int fits64 = 0, fits128 = 0;
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = lt::kDecodeMaxSplits;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(lt::kDecodeMaxSplits, 1, 1);
+      cfg.blockDim = dim3(lt::kDecodeThreads, 1, 1);
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&fits64, lt::decode_kernel<64>, &cfg) == cudaSuccess &&
+          cudaOccupancyMaxActiveClusters(&fits128, lt::decode_kernel<128>, &cfg) == cudaSuccess && fits64 > 0 &&
+          fits128 > 0)
+        info.max_decode_splits = lt::kDecodeMaxSplits;
+    }
+    cudaGetLastError();   // a refused query above is not an error of a later call
     info.ready = true;
   }
   if (!g_encode) {
@@ -396,6 +421,45 @@ lt_status lt_stream_append(void* K_stream, void* V_stream, int32_t* stream_len, 
   return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
 }
 
+namespace {
+
+// CTAs per (sequence, KV head): a power of two up to the device's cluster
+// limit, at least 128 rows each, and no more CTAs than two per SM in total.
+int decode_splits(const DeviceInfo* dev, int batch, int hkv, int max_len) {
+  int splits = 1;
+  while (splits < dev->max_decode_splits && (long long)batch * hkv * splits * 2 <= 2LL * dev->sm_count &&
+         max_len / (splits * 2) >= 128)
+    splits *= 2;
+  return splits;
+}
+
+lt_status launch_decode(lt::DecodeParams& p, int head_dim, int max_len, float softmax_scale, lt_stream stream) {
+  DeviceInfo* dev = nullptr;
+  lt_status st = device_info(&dev);
+  if (st != LT_OK) return st;
+  p.group = p.hq / p.hkv;
+  p.max_len = max_len;
+  p.splits = decode_splits(dev, p.batch, p.hkv, max_len);
+  p.scale_log2 = resolve_scale(softmax_scale, head_dim) * kLog2e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.hkv * p.splits, p.batch, 1);
+  cfg.blockDim = dim3(lt::kDecodeThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = head_dim == 64 ? cudaLaunchKernelEx(&cfg, lt::decode_kernel<64>, p)
+                                       : cudaLaunchKernelEx(&cfg, lt::decode_kernel<128>, p);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
+}
+
+}  // namespace
+
 lt_status lt_stream_decode(const void* q, const void* K_stream, const void* V_stream, const int32_t* stream_len,
                            int batch, int hq, int hkv, int head_dim, int slots, void* O, float* LSE,
                            float softmax_scale, lt_stream stream) {
@@ -404,29 +468,49 @@ lt_status lt_stream_decode(const void* q, const void* K_stream, const void* V_st
       slots < 1 || !std::isfinite(softmax_scale))
     return LT_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return LT_ERR_UNSUPPORTED;
-  DeviceInfo* dev = nullptr;
-  lt_status st = device_info(&dev);
-  if (st != LT_OK) return st;
-  lt::DecodeParams p;
+  if ((long long)hkv * lt::kDecodeMaxSplits > 2147483647LL) return LT_ERR_INVALID_ARG;
+  lt::DecodeParams p{};
   p.batch = batch;
   p.hq = hq;
   p.hkv = hkv;
-  p.group = hq / hkv;
-  p.slots = slots;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.K = static_cast<const __nv_bfloat16*>(K_stream);
   p.V = static_cast<const __nv_bfloat16*>(V_stream);
+  p.seq_start = nullptr;
+  p.seq_stride = (long long)hkv * slots * head_dim;
+  p.row_stride = head_dim;
+  p.head_stride = (long long)slots * head_dim;
   p.len = stream_len;
   p.O = static_cast<__nv_bfloat16*>(O);
   p.LSE = LSE;
-  p.scale_log2 = resolve_scale(softmax_scale, head_dim) * kLog2e;
-  const dim3 grid(hkv, batch);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (head_dim == 64)
-    lt::stream_decode_kernel<64><<<grid, 128, 0, s>>>(p);
-  else
-    lt::stream_decode_kernel<128><<<grid, 128, 0, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+  return launch_decode(p, head_dim, slots, softmax_scale, stream);
+}
+
+lt_status lt_decode_attn(const void* q, const void* K, const void* V, const int32_t* seq_start, int seq_capacity,
+                         const int32_t* len, int batch, int hq, int hkv, int head_dim, int max_len, void* O,
+                         float* LSE, float softmax_scale, lt_stream stream) {
+  if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(len, 4) || !aligned(O, 16) ||
+      !aligned(LSE, 4) || (seq_start && !aligned(seq_start, 4)) || batch < 1 || batch > 65535 || hq < 1 ||
+      hkv < 1 || hq % hkv || max_len < 1 || (!seq_start && seq_capacity < max_len) ||
+      !std::isfinite(softmax_scale))
+    return LT_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return LT_ERR_UNSUPPORTED;
+  if ((long long)hkv * lt::kDecodeMaxSplits > 2147483647LL) return LT_ERR_INVALID_ARG;
+  lt::DecodeParams p{};
+  p.batch = batch;
+  p.hq = hq;
+  p.hkv = hkv;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.K = static_cast<const __nv_bfloat16*>(K);
+  p.V = static_cast<const __nv_bfloat16*>(V);
+  p.seq_start = seq_start;
+  p.row_stride = (long long)hkv * head_dim;
+  p.seq_stride = seq_start ? 0 : (long long)seq_capacity * p.row_stride;
+  p.head_stride = head_dim;
+  p.len = len;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.LSE = LSE;
+  return launch_decode(p, head_dim, max_len, softmax_scale, stream);
 }
 
 lt_status lt_selftest_wait_timeout(unsigned limit_us, lt_stream stream) {

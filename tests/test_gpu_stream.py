@@ -1,9 +1,8 @@
-"""Streaming-attention decode on a demoted layer's cache: against the fp64
+"""Decode attention: on a demoted layer's streaming cache against the fp64
 oracle, against the prefill through the identity
     log sum_{j in K_i} exp(s_ij) = LSE_i + log r_i,
-and the ring-buffer append against a Python model of it."""
-import math
-
+the ring-buffer append against a Python model of it; and on a kept layer's
+full cache against the oracle and against the prefill's last row."""
 import numpy as np
 import pytest
 import torch
@@ -160,3 +159,73 @@ def test_stream_rejects_bad_args():
     nxt = torch.zeros(1, dtype=torch.int32, device="cuda")
     with pytest.raises(lt.LtError):
         lt.lt_stream_ring_init(ln, nxt, 4, 0)
+
+
+def oracle_decode_full(q, K, V, starts, ln):
+    """Oracle of lt_decode_attn on a token-major cache K/V [rows, hkv, d]."""
+    B, hq, d = q.shape
+    hkv = K.shape[1]
+    g = hq // hkv
+    m_max = max(1, int(max(ln)))
+    kb, vb = synth.bf16_bits(K), synth.bf16_bits(V)
+    items_k = np.zeros((B * hq, m_max, d), np.uint16)
+    items_v = np.zeros((B * hq, m_max, d), np.uint16)
+    for b in range(B):
+        n = int(ln[b])
+        for h in range(hq):
+            items_k[b * hq + h, :n] = kb[starts[b]:starts[b] + n, h // g]
+            items_v[b * hq + h, :n] = vb[starts[b]:starts[b] + n, h // g]
+    m = np.repeat(np.asarray(ln, np.int32), hq)
+    O, LSE = oracle.attn_keys(synth.bf16_bits(q).reshape(B * hq, d), items_k, items_v, m)
+    return O.reshape(B, hq, d), LSE.reshape(B, hq)
+
+
+@pytest.mark.parametrize("spec", [dict(seqlens=(300, 37, 1500), hq=8, hkv=2, d=64),
+                                  dict(seqlens=(129, 2000), hq=10, hkv=2, d=128),
+                                  dict(seqlens=(4096,), hq=32, hkv=8, d=64)], ids=["ragged-d64", "d128-g5", "4k"])
+def test_full_decode_of_last_row_equals_prefill(spec):
+    """Decoding each sequence's last prefill query over the packed prefill K/V
+    gives the prefill's own last-row O and LSE (the last row sees every key)."""
+    cfg = synth.custom(seqlens=spec["seqlens"], hq=spec["hq"], hkv=spec["hkv"], d=spec["d"], S=4, W=64, n_obs=8,
+                       seed=17)
+    Q, K, V = synth.layer_inputs(cfg, 0, "cuda")
+    O_pf, LSE_pf = gpu_attention(cfg, Q, K, V)
+    cu_h = np.array(cfg.cu_seqlens(), np.int32)
+    starts = torch.tensor(cu_h[:-1], dtype=torch.int32, device="cuda")
+    ln = torch.tensor(np.diff(cu_h), dtype=torch.int32, device="cuda")
+    last = torch.tensor(cu_h[1:] - 1, device="cuda", dtype=torch.long)
+    q = Q[last].contiguous()
+    O, L = lt.lt_decode_attn(q, K, V, ln, seq_start=starts, max_len=cfg.max_seqlen)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle_decode_full(q, K, V, cu_h[:-1], np.diff(cu_h))
+    compare(O, L, O_ref, L_ref)
+    # Same numbers as the prefill kernel's last rows.
+    assert (L - LSE_pf[:, last].T).abs().max().item() <= 2 * LSE_ABS
+    diff = (O.float() - O_pf[last].float()).norm() / O_pf[last].float().norm()
+    assert diff.item() <= 2 * O_REL_L2
+
+
+@pytest.mark.parametrize("B,cap,hq,hkv,d", [(6, 300, 8, 2, 64), (3, 20000, 8, 8, 128), (2, 70, 6, 3, 128),
+                                             (1, 9000, 16, 8, 64)])
+def test_full_decode_padded_cache_matches_oracle(B, cap, hq, hkv, d):
+    g = torch.Generator(device="cuda").manual_seed(cap + d)
+    q = torch.randn((B, hq, d), generator=g, device="cuda").bfloat16()
+    K = (torch.randn((B, cap, hkv, d), generator=g, device="cuda") * 1.2).bfloat16()
+    V = torch.randn((B, cap, hkv, d), generator=g, device="cuda").bfloat16()
+    lens = [cap, 0, 1, cap // 3, cap - 1, 129][:B]
+    ln = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    O, L = lt.lt_decode_attn(q, K, V, ln)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle_decode_full(q, K.reshape(B * cap, hkv, d), V.reshape(B * cap, hkv, d),
+                                      [b * cap for b in range(B)], lens)
+    compare(O, L, O_ref, L_ref)
+
+
+def test_full_decode_rejects_bad_args():
+    q = torch.zeros((2, 4, 64), dtype=torch.bfloat16, device="cuda")
+    K = torch.zeros((2, 16, 2, 64), dtype=torch.bfloat16, device="cuda")
+    ln = torch.ones(2, dtype=torch.int32, device="cuda")
+    with pytest.raises(lt.LtError):            # capacity below max_len
+        lt.lt_decode_attn(q, K, K, ln, max_len=17)
+    with pytest.raises(ValueError):            # packed cache without seq_start
+        lt.lt_decode_attn(q, K[0], K[0], ln)
