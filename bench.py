@@ -318,6 +318,7 @@ def run_ours(args, cfg, rank, world):
     traffic = recorded_traffic(cfg.name)
     comp_gbs = compaction_bytes(cfg, 1) / t_comp / 1e9
 
+    decode = measure_decode(cfg, lt, pf, peaks)
     e2e = measure_e2e(args, cfg, lt, pf, world)
     cpu = cpu_baseline(cfg) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     clocks = clk.summary()
@@ -355,6 +356,7 @@ def run_ours(args, cfg, rank, world):
         "compaction_gbs": round(comp_gbs, 1),
         "compaction_us_per_layer": round(t_comp * 1e6, 2),
         "device_queue_matches_host_queue": queue_agrees,
+        **decode,
         "roofline": {"kernel": "attn_fwd_kernel (fused with the lazy ratio)", "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": peak_sus, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_sus, 4), "traffic": traffic,
@@ -365,6 +367,90 @@ def run_ours(args, cfg, rank, world):
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
     }
     return line
+
+
+def measure_decode(cfg, lt, pf, peaks):
+    """One decode step (one new query per sequence, every layer) after the
+    prefill: demoted layers read their S+W streaming cache, kept layers their
+    full prefill cache.  Timed against the same step with every layer full.
+    The demotions are sequence 0's (the benchmark workload has batch 1).  Each
+    replay is timed alone with the 126 MB L2 flushed before it."""
+    _, order = pf.dq.result()
+    demoted = [int(x) for x in order[0].tolist() if x >= 0]
+    slot_of = {l: k for k, l in enumerate(demoted)}
+    B, d = cfg.batch, cfg.d
+    g = torch.Generator(device="cuda").manual_seed(5)
+    q = torch.randn((B, cfg.hq, d), generator=g, device="cuda").bfloat16()
+    O = torch.empty_like(q)
+    LSE = torch.empty((B, cfg.hq), dtype=torch.float32, device="cuda")
+    cu_h = cfg.cu_seqlens()
+    starts = torch.tensor(cu_h[:-1], dtype=torch.int32, device="cuda")
+    lens = torch.tensor([cu_h[b + 1] - cu_h[b] for b in range(B)], dtype=torch.int32, device="cuda")
+    stream = torch.cuda.Stream()
+
+    def full(l, s):
+        _, K, V = pf.layers[l]
+        lt.lt_decode_attn(q, K, V, lens, seq_start=starts, max_len=cfg.max_seqlen, out=O, lse=LSE, stream=s)
+
+    def streaming(l, s):
+        k = slot_of[l]
+        lt.lt_stream_decode(q, pf.K_pool[k], pf.V_pool[k], pf.pool_len[k], out=O, lse=LSE, stream=s)
+
+    def hybrid_step(s):
+        for l in range(cfg.layers):
+            (streaming if l in slot_of else full)(l, s)
+
+    def full_step(s):
+        for l in range(cfg.layers):
+            full(l, s)
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
+
+    def timed(fn, reps=10):
+        with torch.cuda.stream(stream):
+            fn(stream)                       # eager warm-up outside capture
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            fn(stream)
+        out = []
+        for r in range(reps + 2):
+            flush.zero_()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+            torch.cuda.synchronize()
+            if r >= 2:
+                out.append(e0.elapsed_time(e1) * 1e-3)
+        return statistics.median(out)
+
+    t_hybrid = timed(hybrid_step)
+    t_full = timed(full_step)
+    t_full_layer = timed(lambda s: full(0, s), reps=20)
+    t_stream_layer = timed(lambda s: streaming(demoted[0], s), reps=20) if demoted else None
+    del flush
+    n_rows = sum(cu_h[b + 1] - cu_h[b] for b in range(B))
+    full_bytes = n_rows * cfg.hkv * d * 2 * 2 + 2 * B * cfg.hq * d * 2 + B * cfg.hq * 4
+    peak_hbm = float(peaks["hbm_gbs"])
+    gbs = full_bytes / t_full_layer / 1e9
+    out = {
+        "decode_layers_streaming": len(demoted),
+        "decode_hybrid_us_per_token": round(t_hybrid * 1e6, 2),
+        "decode_all_full_us_per_token": round(t_full * 1e6, 2),
+        "decode_speedup_vs_all_full": round(t_full / t_hybrid, 3),
+        "decode_full_layer_us": round(t_full_layer * 1e6, 2),
+        "decode_full_layer_gbs": round(gbs, 1),
+        "decode_full_layer_frac_of_hbm": round(gbs / peak_hbm, 4),
+    }
+    if t_stream_layer is not None:
+        slots = cfg.S + cfg.W
+        s_bytes = B * cfg.hkv * min(slots, max(cu_h[b + 1] - cu_h[b] for b in range(B))) * d * 2 * 2
+        out["decode_stream_layer_us"] = round(t_stream_layer * 1e6, 2)
+        out["decode_stream_layer_gbs"] = round(s_bytes / t_stream_layer / 1e9, 1)
+    return out
 
 
 def measure_e2e(args, cfg, lt, pf, world):
