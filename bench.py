@@ -40,7 +40,8 @@ import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "prefill attn+lazy-ratio TFLOP/s & % BF16 tensor peak; compaction GB/s; ratio ovh %"
-ATTN_SOURCES = ["kv_cache_compression_tcgen05_b200/csrc/attn_fwd.cuh", "kv_cache_compression_tcgen05_b200/csrc/lt_device.cuh"]
+ATTN_SOURCES = ["kv_cache_compression_tcgen05_b200/csrc/attn_fwd64.cuh", "kv_cache_compression_tcgen05_b200/csrc/attn_fwd.cuh",
+                "kv_cache_compression_tcgen05_b200/csrc/lt_device.cuh"]
 
 
 def load_peaks():
@@ -63,7 +64,7 @@ def source_digest(paths):
 def recorded_traffic(config_name):
     """DRAM bytes per attention launch from the committed ncu summary, or None if
     the kernel source changed since the counters were taken."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_{config_name}.traffic.txt")
+    path = os.path.join(ROOT, "profiles", f"attn_fwd64_{config_name}.traffic.txt")
     if not os.path.exists(path):
         return None
     with open(path) as f:
@@ -357,7 +358,7 @@ def run_ours(args, cfg, rank, world):
         "compaction_us_per_layer": round(t_comp * 1e6, 2),
         "device_queue_matches_host_queue": queue_agrees,
         **decode,
-        "roofline": {"kernel": "attn_fwd_kernel (fused with the lazy ratio)", "bound": "tensor",
+        "roofline": {"kernel": "attn_fwd64_kernel (head_dim 64, fused with the lazy ratio)", "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": peak_sus, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_sus, 4), "traffic": traffic,
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)"},

@@ -4,7 +4,8 @@
 // The LightTransfer write-up (xzbcqc.com news page, first solution of
 // LightTransfer-Test) reuses the log-sum-exp that a FlashAttention-style prefill
 // produces as the denominator of the lazy ratio.  This kernel is that prefill,
-// built for B200:
+// built for B200 (the library runs it at head_dim 128; head_dim 64 runs the
+// variant in attn_fwd64.cuh, whose P has TMEM columns of its own):
 //
 //   * persistent: one CTA per SM walks a list of work items, heaviest first,
 //     snake-ordered across CTAs.  A work item is two 128-row query tiles that

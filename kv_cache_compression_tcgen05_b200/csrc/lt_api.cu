@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "attn_fwd.cuh"
+#include "attn_fwd64.cuh"
 #include "compact_kv.cuh"
 #include "dqueue.cuh"
 #include "lazy_ratio.cuh"
@@ -50,12 +51,12 @@ lt_status device_info(DeviceInfo** out) {
     void* addr = nullptr;
     if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess) return LT_ERR_CUDA;
     info.status = static_cast<unsigned*>(addr);
-    if (cudaFuncSetAttribute(lt::attn_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             lt::AttnLayout<64>::kAlloc) != cudaSuccess ||
+    if (cudaFuncSetAttribute(lt::attn_fwd64_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             lt::Attn64Layout::kAlloc) != cudaSuccess ||
         cudaFuncSetAttribute(lt::attn_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              lt::AttnLayout<128>::kAlloc) != cudaSuccess ||
-        cudaFuncSetAttribute(lt::attn_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             lt::AttnLayout<64>::kAlloc) != cudaSuccess ||
+        cudaFuncSetAttribute(lt::attn_fwd64_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             lt::Attn64Layout::kAlloc) != cudaSuccess ||
         cudaFuncSetAttribute(lt::attn_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              lt::AttnLayout<128>::kAlloc) != cudaSuccess ||
         cudaFuncSetAttribute(lt::lazy_ratio_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -196,11 +197,11 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
   p.n_obs = n_obs;
   const int grid = int(num_items < dev->sm_count ? num_items : dev->sm_count);
   if (d == 64) {
-    constexpr int kThreads = lt::AttnLayout<64>::kThreads, kSmem = lt::AttnLayout<64>::kAlloc;
+    constexpr int kThreads = lt::Attn64Layout::kThreads, kSmem = lt::Attn64Layout::kAlloc;
     if (ratio)
-      lt::attn_fwd_kernel<64, true><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
+      lt::attn_fwd64_kernel<true><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
     else
-      lt::attn_fwd_kernel<64, false><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
+      lt::attn_fwd64_kernel<false><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
   } else {
     constexpr int kThreads = lt::AttnLayout<128>::kThreads, kSmem = lt::AttnLayout<128>::kAlloc;
     if (ratio)

@@ -243,6 +243,25 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x on the FMA and integer pipes, for a share of the softmax exponentials
+// that the MUFU unit would otherwise serialise.  Range reduction by rounding:
+// adding 1.5 * 2^23 leaves round(x) in the low mantissa bits of the sum
+// (IEEE-754 round-to-nearest), so x = n + f with f in [-0.5, 0.5]; 2^f is a
+// cubic whose coefficients were fitted here by least squares on Chebyshev
+// nodes of [-0.5, 0.5] (relative error below 8e-5 there, against the bf16
+// rounding of P at 2^-9); 2^n is added to the exponent field.  Inputs are
+// clamped at -126 (a result of about 1e-38 stands for 0).
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;          // 1.5 * 2^23
+  const float f = x - (t - 12582912.f);    // x - round(x)
+  const float p = fmaf(fmaf(fmaf(0.05508868396282196f, f, 0.24260404706001282f), f, 0.6932762265205383f), f,
+                       0.9999289512634277f);
+  // The low bits of t's representation hold round(x) (two's complement within
+  // the mantissa); shifted by 23 they become round(x) in the exponent field.
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 // max(a, b, c) in one instruction (three-input max of sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
