@@ -362,20 +362,21 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
         // (and with O, before a rescale): within an item that is one phase
         // of pv_done per key tile; the first tile follows the previous
         // item's epilogue, which consumed the last PV's phase.
-        float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float2 sum4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const float2 sl2x2 = make_float2(sl2, sl2), neg_mx2 = make_float2(neg_m, neg_m);
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int c0 = cb * 32 + 2 * c;
-            const float x0 = fmaf(__uint_as_float(sr[c0]), sl2, neg_m);
-            const float x1 = fmaf(__uint_as_float(sr[c0 + 1]), sl2, neg_m);
+            const float2 xx = fma_f32x2(make_float2(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1])), sl2x2,
+                                        neg_mx2);
             // kPolyPairs of every 16 pairs go to the FMA pipe, the rest to MUFU.
             const bool poly = (c & 15) >= 16 - kPolyPairs;
-            const float p0 = poly ? exp2_fma(x0) : fast_exp2(x0);
-            const float p1 = poly ? exp2_fma(x1) : fast_exp2(x1);
-            sum8[c & 7] += p0 + p1;
+            const float p0 = poly ? exp2_fma(xx.x) : fast_exp2(xx.x);
+            const float p1 = poly ? exp2_fma(xx.y) : fast_exp2(xx.y);
+            sum4[c & 3] = add_f32x2(sum4[c & 3], make_float2(p0, p1));
             pk[c] = pack_bf16x2(p0, p1);
           }
           if (cb == 0 && j > 0) {
@@ -386,8 +387,9 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
           tmem_st16(p_col + cb * 16, pk);
         }
         if (!ok) break;
-        const float tile_sum =
-            ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+        const float2 s01 = add_f32x2(sum4[0], sum4[1]), s23 = add_f32x2(sum4[2], sum4[3]);
+        const float2 s0123 = add_f32x2(s01, s23);
+        const float tile_sum = s0123.x + s0123.y;
         l_run += tile_sum;
         if constexpr (kRatio) {
           if (row_obs && qpos - p.W + 1 - j * 128 <= 0) num += tile_sum;
