@@ -14,9 +14,9 @@
 //     [256,320) P of A, [320,384) P of B, [384,448) O of A, [448,512) O of B.
 // The softmax releases S_X(j) as soon as it has loaded it into registers
 // (s_free), so S_X(j+1) = Q_X K_{j+1}^T runs on the tensor core while the
-// softmax exponentiates S_X(j); the softmax writes P_X(j) to TMEM (in
-// chunks, the first one after P_X(j-1) V_{j-1} has finished reading the P
-// columns: pv_done).  Each query tile has its own
+// softmax exponentiates S_X(j); the softmax writes P_X(j) to TMEM in chunks,
+// the first once P_X(j-1) V_{j-1} has finished reading the P columns
+// (pv_done).  Each query tile has its own
 // MMA-issuing thread (warp 1 for tile A, warp 10 for tile B), so the
 // barrier waits and commits of one tile do not delay the other's MMAs.
 // The K/V ring stages and the Q buffers are released by both issuers
@@ -357,13 +357,16 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
             if (part) num += acc;
           }
           }
-        // P_x(j) in four 32-column chunks of bf16 pairs.  Before the first
-        // chunk is written, P_x(j-1) V_{j-1} must be done with the P columns
-        // (and with O, before a rescale): within an item that is one phase
-        // of pv_done per key tile; the first tile follows the previous
-        // item's epilogue, which consumed the last PV's phase.
+        // P_x(j) in four 32-column chunks of bf16 pairs; the first two are
+        // held in registers and written with the third.  Before the first
+        // write, P_x(j-1) V_{j-1} must be done with the P columns (and with O,
+        // before a rescale): within an item that is one phase of pv_done per
+        // key tile; the first tile follows the previous item's epilogue,
+        // which consumed the last PV's phase.  Waiting two chunks in gives
+        // that PV time to finish.
         float2 sum4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float2 sl2x2 = make_float2(sl2, sl2), neg_mx2 = make_float2(neg_m, neg_m);
+        uint32_t pk0[16], pk1[16];
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
           uint32_t pk[16];
@@ -379,12 +382,24 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
             sum4[c & 3] = add_f32x2(sum4[c & 3], make_float2(p0, p1));
             pk[c] = pack_bf16x2(p0, p1);
           }
-          if (cb == 0 && j > 0) {
+          if (cb == 2 && j > 0) {
             ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], cnt_pv & 1, ctl));
             ++cnt_pv;
             tc_fence_after();
           }
-          tmem_st16(p_col + cb * 16, pk);
+          if (cb == 0) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk0[c] = pk[c];
+          } else if (cb == 1) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk1[c] = pk[c];
+          } else {
+            if (cb == 2) {
+              tmem_st16(p_col, pk0);
+              tmem_st16(p_col + 16, pk1);
+            }
+            tmem_st16(p_col + cb * 16, pk);
+          }
         }
         if (!ok) break;
         const float2 s01 = add_f32x2(sum4[0], sum4[1]), s23 = add_f32x2(sum4[2], sum4[3]);
