@@ -308,10 +308,6 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
           tmem_ld32(s_col + 96, c3);
           tmem_wait_ld();
         }
-        // S_x(j) is in registers: its columns may take S_x(j+1).
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[x]);
         if (diag) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
@@ -335,6 +331,10 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
         }
         l_run *= alpha;
         if constexpr (kRatio) num *= alpha;
+        // S_x(j) is in registers: its columns may take S_x(j+1).
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[x]);
         const float neg_m = -m_run;
         if constexpr (kRatio) {
           // Weights of the keys in K_i = [0, min(S, i+1)) U [max(S, i-W+1), i]
