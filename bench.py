@@ -89,6 +89,18 @@ def ratio_flops(cfg):
     return 2.0 * cfg.d * cfg.hq * total
 
 
+def ratio_unique_bytes(cfg):
+    """Bytes the separate ratio pass must touch once per layer: the observed Q
+    rows and their LSE, and the union of the key rows they see (sinks plus the
+    window band of all observed rows)."""
+    total = 0
+    for n in cfg.seqlens:
+        obs = min(cfg.n_obs, n)
+        band = min(n, cfg.S + cfg.W + obs - 1)
+        total += obs * cfg.hq * (2 * cfg.d + 4) + band * cfg.hkv * 2 * cfg.d
+    return total
+
+
 def compaction_bytes(cfg, n_layers):
     """Bytes read + written by compacting n_layers demoted layers (K and V)."""
     rows = sum(min(n, cfg.S + cfg.W) for n in cfg.seqlens)
@@ -231,6 +243,10 @@ def run_ours(args, cfg, rank, world):
     with torch.cuda.stream(stream):
         pf.enqueue_step(stream)           # eager warm-up: per-device set-up happens outside capture
     torch.cuda.synchronize()
+    if args.decode_only:
+        # One prefill step for the demotions, then the decode leg alone (a
+        # short command for profiling the decode kernel).
+        return {"metric": "decode after prefill", "config": cfg.name, **measure_decode(cfg, lt, pf, peaks)}
     g_step = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step, stream=stream):
         pf.enqueue_step(stream)
@@ -307,8 +323,24 @@ def run_ours(args, cfg, rank, world):
             torch.cuda.synchronize()
             if rep > 0:
                 c_times.append(e0.elapsed_time(e1) * 1e-3)
+    # All demoted layers of the step in one launch (the per-layer launch above is latency bound).
+    _, order_now = pf.dq.result()
+    demoted_layers = order_now[0].to(torch.int32).contiguous()
+    n_dem = int((demoted_layers >= 0).sum())
+    cb_times = []
+    for rep in range(6):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        lt.lt_compact_kv_layers(pf.Kp, pf.Vp, demoted_layers, cfg.S, cfg.W, pf.K_pool, pf.V_pool, pf.pool_len,
+                                cfg.total_tokens, cfg.hkv, cfg.d, **kw)
+        e1.record()
+        torch.cuda.synchronize()
+        if rep > 0:
+            cb_times.append(e0.elapsed_time(e1) * 1e-3)
     del flush
     t_comp = statistics.mean(c_times)
+    t_comp_batch = statistics.median(cb_times)
 
     fl_attn, fl_ratio = attention_flops(cfg), ratio_flops(cfg)
     step_flops = cfg.layers * (fl_attn + fl_ratio)
@@ -356,6 +388,9 @@ def run_ours(args, cfg, rank, world):
         "separate_ratio_overhead_pct": round(100 * t_ratio / t_attn, 3),
         "compaction_gbs": round(comp_gbs, 1),
         "compaction_us_per_layer": round(t_comp * 1e6, 2),
+        "compaction_batched_layers": n_dem,
+        "compaction_batched_gbs": round(compaction_bytes(cfg, n_dem) / t_comp_batch / 1e9, 1),
+        "separate_ratio_unique_gbs": round(ratio_unique_bytes(cfg) / t_ratio / 1e9, 1),
         "device_queue_matches_host_queue": queue_agrees,
         **decode,
         "roofline": {"kernel": "attn_fwd64_kernel (head_dim 64, fused with the lazy ratio)", "bound": "tensor",
@@ -605,6 +640,8 @@ def main():
     ap.add_argument("--config", default="gqa1p2b")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="one prefill step, then only the decode measurement (for profiling the decode kernel)")
     ap.add_argument("--kernels-only", action="store_true",
                     help="time only the device steps (no e2e, CPU baseline or compaction leg); for profiling")
     args = ap.parse_args()

@@ -185,6 +185,21 @@ lt_status lt_compact_kv(const lt_shape* shape, const void* K, const void* V, con
                         void* K_stream, void* V_stream, int32_t* stream_len, lt_stream stream);
 
 /*
+ * The same compaction for several layers in one launch, every sequence:
+ *   K_pool[k, b, kh, r, :] = K_{layers[k]}[cu[b] + p_r, kh, :],
+ *   pool_len[k, b] = |p|,  rows r >= |p| zero,  for k < n.
+ * A layer index outside [0, L) leaves slot k untouched.  K_layers, V_layers:
+ * device arrays of L device pointers (layer l's K/V [T, hkv, d] bf16);
+ * layers: device int32 [n], 0 <= n <= L; K_pool, V_pool: device bf16
+ * [n, batch, hkv, S+W, d]; pool_len: device int32 [n, batch].  One layer's
+ * compaction is a few MB and bound by latency; the demoted layers of a whole
+ * prefill together give the copy engine enough independent work.
+ */
+lt_status lt_compact_kv_layers(const lt_shape* shape, const void* const* K_layers, const void* const* V_layers, int L,
+                               const int32_t* layers, int n, int S, int W, void* K_pool, void* V_pool,
+                               int32_t* pool_len, lt_stream stream);
+
+/*
  * Device-resident layer queue (the queue of lt_queue_push kept in device
  * memory, one per sequence of a batch), so that a whole prefill -- attention,
  * ratio, queue, compaction for every layer -- is one stream of kernels with no

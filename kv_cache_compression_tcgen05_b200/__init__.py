@@ -37,6 +37,7 @@ from .binding import (  # noqa: F401
     DeviceQueue,
     layer_pointer_table,
     lt_compact_kv_pending,
+    lt_compact_kv_layers,
     lt_dqueue_error,
     lt_dqueue_init,
     lt_dqueue_push,

@@ -61,6 +61,7 @@ _SIGS = {
     "lt_dqueue_result": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "lt_dqueue_error": (_i, [_vp, ctypes.POINTER(_i)]),
     "lt_compact_kv_pending": (_i, [_shp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "lt_compact_kv_layers": (_i, [_shp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "lt_stream_ring_init": (_i, [_vp, _vp, _i, _i, _i, _vp]),
     "lt_stream_append": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "lt_stream_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp]),
@@ -417,6 +418,29 @@ def lt_compact_kv_pending(K_layers, V_layers, queue, S, W, K_pool, V_pool, pool_
                                            queue.state.data_ptr(), queue.L, queue.budget, int(S), int(W),
                                            K_pool.data_ptr(), V_pool.data_ptr(), pool_len.data_ptr(),
                                            _stream_handle(stream)), "lt_compact_kv_pending")
+
+
+def lt_compact_kv_layers(K_layers, V_layers, layers, S, W, K_pool, V_pool, pool_len, total_tokens, hkv, d,
+                         cu_seqlens=None, max_seqlen=None, stream=None):
+    """Compaction of the layers listed in `layers` (device int32 [n]) into
+    pool slots 0..n-1 in one launch (see include/lt.h).  K_layers / V_layers:
+    device int64 pointer tables from layer_pointer_table."""
+    for t, n in ((K_layers, "K_layers"), (V_layers, "V_layers")):
+        _dev_tensor(t, n, torch.int64, 1)
+    _dev_tensor(layers, "layers", torch.int32, 1)
+    L, n = K_layers.numel(), layers.numel()
+    if V_layers.numel() != L:
+        raise ValueError("K_layers and V_layers must hold the same number of layers")
+    slots = int(S) + int(W)
+    shape = _shape(total_tokens, hkv, hkv, d, cu_seqlens, max_seqlen)
+    for t, nm in ((K_pool, "K_pool"), (V_pool, "V_pool")):
+        _dev_tensor(t, nm, torch.bfloat16, 5)
+        if t.shape != (n, shape.batch, hkv, slots, d):
+            raise ValueError(f"{nm} must be [n, batch, hkv, S+W, d]")
+    _dev_tensor(pool_len, "pool_len", torch.int32, 2)
+    _check(library().lt_compact_kv_layers(ctypes.byref(shape), K_layers.data_ptr(), V_layers.data_ptr(), L,
+                                          layers.data_ptr(), n, int(S), int(W), K_pool.data_ptr(), V_pool.data_ptr(),
+                                          pool_len.data_ptr(), _stream_handle(stream)), "lt_compact_kv_layers")
 
 
 def lt_stream_ring_init(stream_len, next_slot, S, W, stream=None):

@@ -73,4 +73,59 @@ __global__ void __launch_bounds__(256) compact_kv_kernel(const CompactParams p) 
     if (!p.mask[b]) p.len[b] = 0;
 }
 
+// Compaction of several layers in one launch: pool slot k receives the
+// streaming rows of layer layers[k] for every sequence (same gather as
+// compact_kv_kernel with all sequences selected); a layer index outside
+// [0, L) leaves its slot untouched.  Enough independent 16-byte pieces for the
+// whole launch keep HBM busy where one layer alone is bound by latency.
+struct CompactLayersParams {
+  int batch, total_tokens, hkv, D, S, W, L, n;
+  const int32_t* cu_seqlens;
+  const uint4* const* K_layers;   // device array [L] of the layers' K base pointers
+  const uint4* const* V_layers;
+  const int32_t* layers;          // [n]
+  uint4* K_pool;                  // [n, batch, hkv, S+W, d]
+  uint4* V_pool;
+  int32_t* pool_len;              // [n, batch]
+};
+
+__global__ void __launch_bounds__(256) compact_layers_kernel(const CompactLayersParams p) {
+  const int pieces = p.D / 8;
+  const int slots = p.S + p.W;
+  const long long per_seq = (long long)slots * p.hkv * pieces;
+  const long long per_slot = per_seq * p.batch;
+  const long long total = per_slot * p.n;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < total; x += stride) {
+    const int k = int(x / per_slot);
+    const int layer = p.layers[k];
+    if (layer < 0 || layer >= p.L) continue;
+    long long rem = x - (long long)k * per_slot;
+    const int b = int(rem / per_seq);
+    rem -= (long long)b * per_seq;
+    const int r = int(rem / ((long long)p.hkv * pieces));
+    rem -= (long long)r * p.hkv * pieces;
+    const int kh = int(rem / pieces);
+    const int piece = int(rem - (long long)kh * pieces);
+    int start = 0, N = p.total_tokens;
+    if (p.cu_seqlens) {
+      start = p.cu_seqlens[b];
+      N = p.cu_seqlens[b + 1] - start;
+    }
+    const int n_sink = min(p.S, N);
+    const int keep = min(N, slots);
+    const size_t dst = (((size_t(k) * p.batch + b) * p.hkv + kh) * slots + r) * pieces + piece;
+    if (r < keep) {
+      const int pos = r < n_sink ? r : max(p.S, N - p.W) + (r - n_sink);
+      const size_t src = ((size_t(start) + pos) * p.hkv + kh) * pieces + piece;
+      p.K_pool[dst] = p.K_layers[layer][src];
+      p.V_pool[dst] = p.V_layers[layer][src];
+    } else {
+      p.K_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+      p.V_pool[dst] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (r == 0 && kh == 0 && piece == 0) p.pool_len[size_t(k) * p.batch + b] = keep;
+  }
+}
+
 }  // namespace lt

@@ -25,9 +25,10 @@
 // of a warp takes one row at a time, 8 elements per lane in one 16-byte load
 // (the next row's loads in flight while the current one is used), scores are
 // reduced over the group's lanes with shuffles, and each group keeps a running
-// (max, sum, output) per head in the log2 domain.  Groups merge through shuffles, warps through shared memory
-// and the cluster's CTAs through distributed shared memory into CTA rank 0,
-// which writes O and LSE.
+// (max, sum, output) per head in the log2 domain.  Groups merge through
+// shuffles; warps through shared memory and the cluster's CTAs through
+// distributed shared memory, each with one thread per (head, element), rank 0
+// writing O and LSE.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -229,55 +230,47 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
       }
     }
     __syncthreads();
-    // Warp 0, row group 0: merge the warps into the CTA's partial state.
-    if (warp == 0 && rgw == 0) {
+    // Merge the warps into the CTA's partial state: one thread per (head,
+    // element) combines the warps' states against their common maximum.
+    for (int i = threadIdx.x; i < kDecodeHeads * D; i += kDecodeThreads) {
+      const int hh = i / D, e = i - hh * D;
+      float M = -INFINITY;
 #pragma unroll
-      for (int hh = 0; hh < kDecodeHeads; ++hh) {
-        float mm = sm_m[0][hh], ll = sm_l[0][hh], oo[E];
+      for (int w2 = 0; w2 < kDecodeWarps; ++w2) M = fmaxf(M, sm_m[w2][hh]);
+      float ll = 0.f, oo = 0.f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) oo[e] = sm_o[0][hh][li * E + e];
-        for (int w2 = 1; w2 < kDecodeWarps; ++w2) {
-          float o2[E];
-#pragma unroll
-          for (int e = 0; e < E; ++e) o2[e] = sm_o[w2][hh][li * E + e];
-          softmax_merge<E>(mm, ll, oo, sm_m[w2][hh], sm_l[w2][hh], o2);
-        }
-        if (li == 0) {
-          cta_m[hh] = mm;
-          cta_l[hh] = ll;
-        }
-#pragma unroll
-        for (int e = 0; e < E; ++e) cta_o[hh][li * E + e] = oo[e];
+      for (int w2 = 0; w2 < kDecodeWarps; ++w2) {
+        const float c = M == -INFINITY ? 0.f : fast_exp2(sm_m[w2][hh] - M);
+        ll = fmaf(sm_l[w2][hh], c, ll);
+        oo = fmaf(sm_o[w2][hh][e], c, oo);
+      }
+      cta_o[hh][e] = oo;
+      if (e == 0) {
+        cta_m[hh] = M;
+        cta_l[hh] = ll;
       }
     }
     cluster.sync();   // every CTA's partial state is visible cluster-wide
-    // Rank 0, warp 0, row group 0: merge the cluster's CTAs in rank order and
-    // write the result.
-    if (split == 0 && warp == 0 && rgw == 0) {
-#pragma unroll
-      for (int hh = 0; hh < kDecodeHeads; ++hh) {
-        float mm = cta_m[hh], ll = cta_l[hh], oo[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) oo[e] = cta_o[hh][li * E + e];
-        for (int r = 1; r < p.splits; ++r) {
-          const float* rm = cluster.map_shared_rank(&cta_m[0], r);
-          const float* rl = cluster.map_shared_rank(&cta_l[0], r);
-          const float* ro = cluster.map_shared_rank(&cta_o[0][0], r);
-          float o2[E];
-#pragma unroll
-          for (int e = 0; e < E; ++e) o2[e] = ro[hh * D + li * E + e];
-          softmax_merge<E>(mm, ll, oo, rm[hh], rl[hh], o2);
+    // Rank 0: one thread per (head, element) combines the cluster's CTAs (in
+    // distributed shared memory) and writes the result.
+    if (split == 0) {
+      for (int i = threadIdx.x; i < kDecodeHeads * D; i += kDecodeThreads) {
+        const int hh = i / D, e = i - hh * D;
+        if (hh >= nh) continue;
+        float M = -INFINITY;
+        for (int r = 0; r < p.splits; ++r) M = fmaxf(M, cluster.map_shared_rank(&cta_m[0], r)[hh]);
+        float ll = 0.f, oo = 0.f;
+        for (int r = 0; r < p.splits; ++r) {
+          const float mr = cluster.map_shared_rank(&cta_m[0], r)[hh];
+          const float c = M == -INFINITY ? 0.f : fast_exp2(mr - M);
+          ll = fmaf(cluster.map_shared_rank(&cta_l[0], r)[hh], c, ll);
+          oo = fmaf(cluster.map_shared_rank(&cta_o[0][0], r)[hh * D + e], c, oo);
         }
-        if (hh < nh) {
-          const int h = kh * p.group + h0 + hh;
-          const float inv = ll > 0.f ? 1.f / ll : 0.f;
-          __nv_bfloat16* orow = p.O + (size_t(b) * p.hq + h) * D + li * E;
-#pragma unroll
-          for (int e = 0; e < E; e += 2)
-            *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(oo[e] * inv, oo[e + 1] * inv);
-          if (li == 0)
-            p.LSE[size_t(b) * p.hq + h] = ll > 0.f ? (mm + fast_log2(ll)) * 0.69314718055994531f : -INFINITY;
-        }
+        const int h = kh * p.group + h0 + hh;
+        const float inv = ll > 0.f ? 1.f / ll : 0.f;
+        p.O[(size_t(b) * p.hq + h) * D + e] = __float2bfloat16_rn(oo * inv);
+        if (e == 0)
+          p.LSE[size_t(b) * p.hq + h] = ll > 0.f ? (M + fast_log2(ll)) * 0.69314718055994531f : -INFINITY;
       }
     }
     cluster.sync();   // rank 0 is done reading before any CTA's state is reused or released

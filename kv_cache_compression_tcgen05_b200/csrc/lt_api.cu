@@ -314,6 +314,43 @@ lt_status lt_compact_kv(const lt_shape* shape, const void* K, const void* V, con
   return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
 }
 
+lt_status lt_compact_kv_layers(const lt_shape* shape, const void* const* K_layers, const void* const* V_layers, int L,
+                               const int32_t* layers, int n, int S, int W, void* K_pool, void* V_pool,
+                               int32_t* pool_len, lt_stream stream) {
+  lt_status st = check_shape(shape);
+  if (st != LT_OK) return st;
+  if (L < 1 || n < 0 || n > L || !aligned(K_layers, 8) || !aligned(V_layers, 8) ||
+      (n > 0 && (!aligned(layers, 4) || !aligned(K_pool, 16) || !aligned(V_pool, 16) || !aligned(pool_len, 4))))
+    return LT_ERR_INVALID_ARG;
+  if (S < 0 || W < 0 || (long long)S + W < 1 || (long long)S + W > (1 << 24)) return LT_ERR_INVALID_ARG;
+  if (n == 0) return LT_OK;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != LT_OK) return st;
+  lt::CompactLayersParams p;
+  p.batch = shape->batch;
+  p.total_tokens = shape->total_tokens;
+  p.hkv = shape->hkv;
+  p.D = shape->head_dim;
+  p.S = S;
+  p.W = W;
+  p.L = L;
+  p.n = n;
+  p.cu_seqlens = shape->cu_seqlens;
+  p.K_layers = reinterpret_cast<const uint4* const*>(K_layers);
+  p.V_layers = reinterpret_cast<const uint4* const*>(V_layers);
+  p.layers = layers;
+  p.K_pool = static_cast<uint4*>(K_pool);
+  p.V_pool = static_cast<uint4*>(V_pool);
+  p.pool_len = pool_len;
+  const long long work = (long long)n * shape->batch * (S + W) * shape->hkv * (shape->head_dim / 8);
+  long long blocks = (work + 255) / 256;
+  const long long cap = (long long)dev->sm_count * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  lt::compact_layers_kernel<<<int(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
 size_t lt_dqueue_state_bytes(int L, int batch) {
   if (L < 1 || batch < 1) return 0;
   return lt::dqueue_bytes(L, batch);

@@ -168,3 +168,32 @@ def test_graph_captured_tiny_prefill():
         Q, K, _ = layers[l]
         ref = oracle.lazy_ratio(cu_h, synth.bf16_bits(Q), synth.bf16_bits(K), cfg.S, cfg.W, cfg.n_obs)
         assert np.abs(ratio[l].cpu().numpy() - ref).max() <= 2e-3
+
+
+def test_compact_kv_layers_matches_oracle():
+    """Several layers compacted in one launch equal the oracle's per-layer
+    compaction; a slot whose layer index is -1 is left untouched."""
+    cfg = synth.custom(layers=5, seqlens=(300, 41, 1000, 7), hq=4, hkv=2, d=128, S=4, W=60, seed=37)
+    layers = [synth.layer_inputs(cfg, l, "cuda") for l in range(cfg.layers)]
+    Kp = lt.layer_pointer_table([lay[1] for lay in layers])
+    Vp = lt.layer_pointer_table([lay[2] for lay in layers])
+    pick = [3, -1, 0, 4]
+    slots = cfg.S + cfg.W
+    K_pool = torch.full((len(pick), cfg.batch, cfg.hkv, slots, cfg.d), -5.0, dtype=torch.bfloat16, device="cuda")
+    V_pool = K_pool.clone()
+    pool_len = torch.full((len(pick), cfg.batch), -7, dtype=torch.int32, device="cuda")
+    cu = torch.tensor(cfg.cu_seqlens(), dtype=torch.int32, device="cuda")
+    lt.lt_compact_kv_layers(Kp, Vp, torch.tensor(pick, dtype=torch.int32, device="cuda"), cfg.S, cfg.W, K_pool, V_pool,
+                            pool_len, cfg.total_tokens, cfg.hkv, cfg.d, cu_seqlens=cu, max_seqlen=cfg.max_seqlen)
+    torch.cuda.synchronize()
+    cu_h = np.array(cfg.cu_seqlens(), np.int32)
+    ones = np.ones(cfg.batch, np.uint8)
+    for k, m in enumerate(pick):
+        if m < 0:
+            assert bool((K_pool[k] == -5.0).all()) and bool((pool_len[k] == -7).all())
+            continue
+        oks, ovs, oln = oracle.compact_kv(cu_h, synth.bf16_bits(layers[m][1]), synth.bf16_bits(layers[m][2]), ones,
+                                          cfg.S, cfg.W)
+        assert np.array_equal(synth.bf16_bits(K_pool[k]), oks)
+        assert np.array_equal(synth.bf16_bits(V_pool[k]), ovs)
+        assert np.array_equal(pool_len[k].cpu().numpy(), oln)
