@@ -219,6 +219,10 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // The set-up above touches no global memory: it overlaps the previous
+  // kernel's tail under a programmatic launch.
+  pdl_wait();
+  pdl_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const WaitCtl ctl{abort_flag, p.status};
   const WaitCtl drain_ctl{no_abort, p.status};

@@ -58,6 +58,8 @@ __host__ __device__ inline DQueueView dqueue_view(void* state, int L, int batch)
 }
 
 __global__ void dqueue_init_kernel(void* state, int L, int budget, int batch) {
+  pdl_wait();
+  pdl_launch_dependents();
   DQueueView v = dqueue_view(state, L, batch);
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   if (tid == 0) {
@@ -81,6 +83,8 @@ __device__ __forceinline__ bool dq_outranks(float sa, int a, float sb, int b) { 
 // in double, as the host lt_layer_score does), push, pop the best-ranked
 // layer while more than C = L - budget are queued.
 __global__ void dqueue_push_kernel(void* state, int L, int batch, int layer, const float* ratio, int hq) {
+  pdl_wait();
+  pdl_launch_dependents();
   DQueueView v = dqueue_view(state, L, batch);
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= batch) return;
@@ -150,6 +154,8 @@ struct CompactPendingParams {
 // k = its demotion index; rows past the kept count are zero.  Same data
 // movement as compact_kv_kernel, with the layer chosen on the device.
 __global__ void __launch_bounds__(256) compact_pending_kernel(const CompactPendingParams p) {
+  pdl_wait();
+  pdl_launch_dependents();
   DQueueView v = dqueue_view(const_cast<void*>(p.state), p.L, p.batch);
   const int pieces = p.D / 8;
   const int slots = p.S + p.W;
@@ -186,6 +192,14 @@ __global__ void __launch_bounds__(256) compact_pending_kernel(const CompactPendi
     }
     if (r == 0 && kh == 0 && piece == 0) p.pool_len[size_t(k) * p.batch + b] = keep;
   }
+}
+
+// Zeroes n floats (the fused ratio's accumulator) as a kernel, so that it can
+// be launched programmatically ahead of the attention.
+__global__ void zero_f32_kernel(float* x, int n) {
+  pdl_wait();
+  pdl_launch_dependents();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) x[i] = 0.f;
 }
 
 }  // namespace lt

@@ -10,6 +10,7 @@
 #include <climits>
 #include <cmath>
 #include <mutex>
+#include <utility>
 
 #include "attn_fwd.cuh"
 #include "attn_fwd64.cuh"
@@ -130,6 +131,26 @@ lt_status make_map(CUtensorMap* map, const void* base, int d, int heads, int T) 
   return r == CUDA_SUCCESS ? LT_OK : LT_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialization: the kernel may be launched
+// while the previous kernel in the stream is finishing; it waits (pdl_wait)
+// before touching memory the previous kernel may use.  Used for the kernels of
+// the prefill loop, whose launch gaps are otherwise a few microseconds each.
+template <typename... ExpTypes, typename... ActTypes>
+cudaError_t launch_pdl(void (*kernel)(ExpTypes...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       ActTypes&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<ActTypes>(args)...);
+}
+
 float resolve_scale(float softmax_scale, int d) {
   return softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(d));
 }
@@ -159,7 +180,8 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
   if (ratio) {
     // The kernel adds each tile's share of the mean; sequences without tokens keep 0.
     if ((st = device_info(&dev)) != LT_OK) return st;
-    if (cudaMemsetAsync(ratio, 0, sizeof(float) * size_t(shape->batch) * shape->hq, s) != cudaSuccess)
+    const int n = shape->batch * shape->hq;
+    if (launch_pdl(lt::zero_f32_kernel, dim3((n + 255) / 256), dim3(256), 0, s, ratio, n) != cudaSuccess)
       return LT_ERR_CUDA;
   }
   if (T == 0 || max_len == 0) return LT_OK;  // nothing to read or write
@@ -196,20 +218,21 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
   p.W = W;
   p.n_obs = n_obs;
   const int grid = int(num_items < dev->sm_count ? num_items : dev->sm_count);
+  cudaError_t e;
   if (d == 64) {
     constexpr int kThreads = lt::Attn64Layout::kThreads, kSmem = lt::Attn64Layout::kAlloc;
     if (ratio)
-      lt::attn_fwd64_kernel<true><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
+      e = launch_pdl(lt::attn_fwd64_kernel<true>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p);
     else
-      lt::attn_fwd64_kernel<false><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
+      e = launch_pdl(lt::attn_fwd64_kernel<false>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p);
   } else {
     constexpr int kThreads = lt::AttnLayout<128>::kThreads, kSmem = lt::AttnLayout<128>::kAlloc;
     if (ratio)
-      lt::attn_fwd_kernel<128, true><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
+      e = launch_pdl(lt::attn_fwd_kernel<128, true>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p);
     else
-      lt::attn_fwd_kernel<128, false><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, p);
+      e = launch_pdl(lt::attn_fwd_kernel<128, false>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p);
   }
-  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
 }
 
 lt_status lt_prefill_attn(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O, float* LSE,
@@ -367,16 +390,16 @@ lt_status lt_dqueue_init(void* state, int L, int budget, int batch, lt_stream st
   DeviceInfo* dev = nullptr;
   lt_status st = device_info(&dev);
   if (st != LT_OK) return st;
-  lt::dqueue_init_kernel<<<dq_blocks(batch), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(state, L, budget,
-                                                                                               batch);
-  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+  const cudaError_t e = launch_pdl(lt::dqueue_init_kernel, dim3(dq_blocks(batch)), dim3(128), 0,
+                                   reinterpret_cast<cudaStream_t>(stream), state, L, budget, batch);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
 }
 
 lt_status lt_dqueue_push(void* state, int L, int batch, int layer, const float* ratio, int hq, lt_stream stream) {
   if (!dq_args(state, L, batch) || !aligned(ratio, 4) || hq < 1) return LT_ERR_INVALID_ARG;
-  lt::dqueue_push_kernel<<<dq_blocks(batch), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(state, L, batch,
-                                                                                               layer, ratio, hq);
-  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+  const cudaError_t e = launch_pdl(lt::dqueue_push_kernel, dim3(dq_blocks(batch)), dim3(128), 0,
+                                   reinterpret_cast<cudaStream_t>(stream), state, L, batch, layer, ratio, hq);
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
 }
 
 lt_status lt_dqueue_result(const void* state, int L, int batch, int budget, uint8_t* lazy_mask, int32_t* order,
@@ -429,7 +452,9 @@ lt_status lt_compact_kv_pending(const lt_shape* shape, const void* const* K_laye
   const long long cap = (long long)dev->sm_count * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  lt::compact_pending_kernel<<<int(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  if (launch_pdl(lt::compact_pending_kernel, dim3(int(blocks)), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream),
+                 p) != cudaSuccess)
+    return LT_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
 }
 

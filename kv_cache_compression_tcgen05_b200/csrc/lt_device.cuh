@@ -83,6 +83,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Programmatic dependent launch.  pdl_wait: wait until the kernel before this
+// one in the stream has completed and its writes are visible (a no-op when the
+// launch was not programmatic); called before a kernel's first access to
+// global memory that the previous kernel may touch.  pdl_launch_dependents:
+// the next kernel may be launched now (its CTAs start when resources free and
+// then wait in pdl_wait), so its launch overlaps this kernel's tail.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ----------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
