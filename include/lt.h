@@ -121,6 +121,16 @@ lt_status lt_prefill_attn_ratio(const lt_shape* shape, const void* Q, const void
                                 lt_stream stream);
 
 /*
+ * lt_prefill_attn_ratio without the zeroing: the kernel adds each query
+ * tile's share of ratio[b, h] to what the buffer holds, so ratio must be zero
+ * on entry (e.g. all layers' ratios cleared by one memset per prefill, instead
+ * of one zeroing launch per layer).  Otherwise identical.
+ */
+lt_status lt_prefill_attn_ratio_acc(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
+                                    float* LSE, float softmax_scale, int S, int W, int n_obs, float* ratio,
+                                    lt_stream stream);
+
+/*
  * Lazy ratio from the LSE.
  *   For every sequence b (length N), query head h and each of the last
  *   n' = min(n_obs, N) rows i of b:

@@ -47,6 +47,7 @@ _shp = ctypes.POINTER(LtShape)
 _SIGS = {
     "lt_prefill_attn": (_i, [_shp, _vp, _vp, _vp, _vp, _vp, _f, _vp]),
     "lt_prefill_attn_ratio": (_i, [_shp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
+    "lt_prefill_attn_ratio_acc": (_i, [_shp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
     "lt_lazy_ratio": (_i, [_shp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
     "lt_layer_score": (_f, [_vp, _i]),
     "lt_select_layers": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
@@ -172,9 +173,12 @@ def lt_prefill_attn(Q, K, V, cu_seqlens=None, max_seqlen=None, softmax_scale=Non
 
 
 def lt_prefill_attn_ratio(Q, K, V, S, W, n_obs, cu_seqlens=None, max_seqlen=None, softmax_scale=None, out=None,
-                          lse=None, ratio=None, stream=None):
+                          lse=None, ratio=None, stream=None, accumulate=False):
     """Attention fused with the lazy ratio.  Returns (O [T, hq, d] bf16,
-    LSE [hq, T] fp32, ratio [batch, hq] fp32)."""
+    LSE [hq, T] fp32, ratio [batch, hq] fp32).  accumulate=True adds into a
+    ratio buffer the caller has zeroed (no zeroing launch)."""
+    if accumulate and ratio is None:
+        raise ValueError("accumulate=True needs a zeroed ratio buffer")
     _dev_tensor(Q, "Q", torch.bfloat16, 3)
     _dev_tensor(K, "K", torch.bfloat16, 3)
     _dev_tensor(V, "V", torch.bfloat16, 3)
@@ -194,7 +198,8 @@ def lt_prefill_attn_ratio(Q, K, V, S, W, n_obs, cu_seqlens=None, max_seqlen=None
     _dev_tensor(ratio, "ratio", torch.float32, 2)
     if out.shape != Q.shape or lse.shape != (hq, T) or ratio.shape != (shape.batch, hq):
         raise ValueError("out must be [T, hq, d], lse [hq, T] and ratio [batch, hq]")
-    _check(library().lt_prefill_attn_ratio(ctypes.byref(shape), Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+    fn = library().lt_prefill_attn_ratio_acc if accumulate else library().lt_prefill_attn_ratio
+    _check(fn(ctypes.byref(shape), Q.data_ptr(), K.data_ptr(), V.data_ptr(),
                                            out.data_ptr(), lse.data_ptr(),
                                            0.0 if softmax_scale is None else float(softmax_scale), int(S), int(W),
                                            int(n_obs), ratio.data_ptr(), _stream_handle(stream)),

@@ -165,7 +165,7 @@ extern "C" {
 // launch.  `ratio` null selects the plain attention kernel.
 static lt_status launch_attention(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
                                   float* LSE, float softmax_scale, int S, int W, int n_obs, float* ratio,
-                                  lt_stream stream) {
+                                  lt_stream stream, bool zero_ratio = true) {
   lt_status st = check_shape(shape);
   if (st != LT_OK) return st;
   if (!std::isfinite(softmax_scale)) return LT_ERR_INVALID_ARG;
@@ -177,7 +177,7 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
   if (T > 0 && (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || !aligned(LSE, 4)))
     return LT_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
-  if (ratio) {
+  if (ratio && zero_ratio) {
     // The kernel adds each tile's share of the mean; sequences without tokens keep 0.
     if ((st = device_info(&dev)) != LT_OK) return st;
     const int n = shape->batch * shape->hq;
@@ -245,6 +245,13 @@ lt_status lt_prefill_attn_ratio(const lt_shape* shape, const void* Q, const void
                                 lt_stream stream) {
   if (!ratio) return LT_ERR_INVALID_ARG;
   return launch_attention(shape, Q, K, V, O, LSE, softmax_scale, S, W, n_obs, ratio, stream);
+}
+
+lt_status lt_prefill_attn_ratio_acc(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
+                                    float* LSE, float softmax_scale, int S, int W, int n_obs, float* ratio,
+                                    lt_stream stream) {
+  if (!ratio) return LT_ERR_INVALID_ARG;
+  return launch_attention(shape, Q, K, V, O, LSE, softmax_scale, S, W, n_obs, ratio, stream, false);
 }
 
 lt_status lt_lazy_ratio(const lt_shape* shape, const void* Q, const void* K, const float* LSE, float softmax_scale,

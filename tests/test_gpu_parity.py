@@ -310,3 +310,25 @@ def test_fused_ratio_full_size(name):
     _, _, r3 = gpu_fused(cfg, Q, K, V)
     torch.cuda.synchronize()
     assert torch.equal(r, r3)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fused_ratio_accumulate_mode(d):
+    """lt_prefill_attn_ratio_acc adds into the caller's buffer: on a zeroed
+    buffer it equals the zeroing call bit for bit, on a buffer holding c it
+    gives c + ratio, and O / LSE are the same."""
+    cfg = synth.custom(seqlens=(300, 77, 513), hq=4, hkv=2, d=d, S=4, W=60, n_obs=16, seed=61)
+    Q, K, V = synth.layer_inputs(cfg, 0, "cuda")
+    cu = torch.tensor(cfg.cu_seqlens(), dtype=torch.int32, device="cuda")
+    kw = dict(cu_seqlens=cu, max_seqlen=cfg.max_seqlen)
+    O1, L1, r1 = lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, **kw)
+    r0 = torch.zeros_like(r1)
+    O2, L2, r2 = lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, ratio=r0, accumulate=True, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(r1, r2) and torch.equal(O1, O2) and torch.equal(L1, L2)
+    rc = torch.full_like(r1, 0.25)
+    lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, ratio=rc, accumulate=True, **kw)
+    torch.cuda.synchronize()
+    assert (rc - (r1 + 0.25)).abs().max().item() <= 1e-6
+    with pytest.raises(ValueError):
+        lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, accumulate=True, **kw)
