@@ -157,3 +157,50 @@ def test_queue_rejects_bad_pushes():
     assert len(q) == 1
     with pytest.raises(lt.LtError):
         lt.lt_queue_create(3, 4)
+
+
+def test_fused_accumulate_and_decode_calls_reject_bad_arguments():
+    """The newer entry points check their arguments before any device call."""
+    lib = lt.library()
+    s = _shape()
+    INV, UNS = lt.LT_ERR_INVALID_ARG, lt.LT_ERR_UNSUPPORTED
+    # fused attention in accumulate mode needs a ratio buffer
+    assert lib.lt_prefill_attn_ratio_acc(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, 0.0, 4, 32, 16, None,
+                                         None) == INV
+    # decode over a full cache: (q, K, V, seq_start, seq_capacity, len, batch, hq, hkv, d, max_len, O, LSE, scale)
+    assert lib.lt_decode_attn(FAKE, FAKE, FAKE, None, 16, FAKE, 1, 4, 2, 64, 17, FAKE, FAKE, 0.0, None) == INV
+    assert lib.lt_decode_attn(FAKE, FAKE, FAKE, None, 16, FAKE, 1, 5, 2, 64, 16, FAKE, FAKE, 0.0, None) == INV
+    assert lib.lt_decode_attn(FAKE, FAKE, FAKE, None, 16, FAKE, 1, 4, 2, 64, 0, FAKE, FAKE, 0.0, None) == INV
+    assert lib.lt_decode_attn(FAKE + 8, FAKE, FAKE, None, 16, FAKE, 1, 4, 2, 64, 16, FAKE, FAKE, 0.0, None) == INV
+    assert lib.lt_decode_attn(FAKE, FAKE, FAKE, None, 16, FAKE, 1, 4, 2, 96, 16, FAKE, FAKE, 0.0, None) == UNS
+    # decode over a streaming cache: (q, K, V, len, batch, hq, hkv, d, slots, O, LSE, scale)
+    assert lib.lt_stream_decode(FAKE, FAKE, FAKE, FAKE, 0, 4, 2, 64, 8, FAKE, FAKE, 0.0, None) == INV
+    assert lib.lt_stream_decode(FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 64, 0, FAKE, FAKE, 0.0, None) == INV
+    assert lib.lt_stream_decode(FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 80, 8, FAKE, FAKE, 0.0, None) == UNS
+    assert lib.lt_stream_decode(FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 64, 8, FAKE, FAKE, float("inf"), None) == INV
+    # ring state
+    assert lib.lt_stream_ring_init(FAKE, FAKE, 1, 4, 0, None) == INV
+    assert lib.lt_stream_ring_init(FAKE + 2, FAKE, 1, 4, 8, None) == INV
+    assert lib.lt_stream_append(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 96, 4, 8, None) == UNS
+
+
+def test_queue_and_pool_calls_reject_bad_arguments():
+    lib = lt.library()
+    s = _shape()
+    INV = lt.LT_ERR_INVALID_ARG
+    assert lib.lt_dqueue_state_bytes(0, 1) == 0 and lib.lt_dqueue_state_bytes(4, 0) == 0
+    assert lib.lt_dqueue_state_bytes(4, 2) > 0
+    assert lib.lt_dqueue_init(FAKE, 4, 5, 1, None) == INV           # budget > L
+    assert lib.lt_dqueue_init(FAKE + 4, 4, 2, 1, None) == INV       # state not 16-byte aligned
+    assert lib.lt_dqueue_push(FAKE, 0, 1, 0, FAKE, 2, None) == INV   # L < 1
+    assert lib.lt_dqueue_push(FAKE, 4, 1, 0, FAKE, 0, None) == INV   # hq < 1
+    # (shape, K_layers, V_layers, state, L, budget, S, W, K_pool, V_pool, pool_len)
+    assert lib.lt_compact_kv_pending(ctypes.byref(s), FAKE, FAKE, FAKE, 4, 0, 4, 8, FAKE, FAKE, FAKE, None) == INV
+    assert lib.lt_compact_kv_pending(ctypes.byref(s), FAKE, FAKE, FAKE, 4, 2, 0, 0, FAKE, FAKE, FAKE, None) == INV
+    # (shape, K_layers, V_layers, L, layers, n, S, W, K_pool, V_pool, pool_len)
+    assert lib.lt_compact_kv_layers(ctypes.byref(s), FAKE, FAKE, 4, FAKE, 5, 4, 8, FAKE, FAKE, FAKE, None) == INV
+    assert lib.lt_compact_kv_layers(ctypes.byref(s), FAKE, FAKE, 0, FAKE, 0, 4, 8, FAKE, FAKE, FAKE, None) == INV
+    assert lib.lt_compact_kv_layers(ctypes.byref(s), FAKE, FAKE, 4, FAKE, 1, 0, 0, FAKE, FAKE, FAKE, None) == INV
+    # nothing to compact: succeeds without a device
+    assert lib.lt_compact_kv_layers(ctypes.byref(s), FAKE, FAKE, 4, None, 0, 4, 8, None, None, None, None) == lt.LT_OK
+    assert lib.lt_selftest_wait_timeout(0, None) == INV
