@@ -14,12 +14,17 @@ attention (lt_prefill_attn), the separate ratio pass from the LSE
 it.
 
 Rank 0 prints one JSON line.  With --gpus N > 1 (torchrun) every rank runs an
-independent replica of the workload (the path has no exchange step): weak
-scaling, value = work of all ranks / max-over-ranks device time.
+independent replica of the workload by default (--shard replicas): weak
+scaling, value = work of all ranks / max-over-ranks device time.  With
+--shard heads the ranks split ONE prefill by KV heads and all-gather the
+per-head ratios of every layer (NCCL, inside the step's graph) before the
+queue push: strong scaling, value = work of the one prefill / max-over-ranks
+device time; per-kernel figures are then those of this rank's head slice.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -157,18 +162,25 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, need_group=False):
+    """One process per GPU; a NCCL process group when several ranks run, or
+    when the heads are split (a single rank then still takes the collective
+    path)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world != n_gpus:
         raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
-    if world > 1:
+    torch.cuda.set_device(local if world > 1 else 0)
+    if world > 1 or need_group:
         import datetime
-        torch.cuda.set_device(local)
+        if world == 1 and "MASTER_ADDR" not in os.environ:
+            import socket
+            with socket.socket() as sock:
+                sock.bind(("127.0.0.1", 0))
+                port = sock.getsockname()[1]
+            os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK="0", WORLD_SIZE="1")
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    else:
-        torch.cuda.set_device(0)
     return rank, world, local
 
 
@@ -189,59 +201,46 @@ def barrier(world):
 # ------------------------------------------------------------------ our arm
 
 class Prefill:
-    """The whole path over every layer of one prefill, inputs resident on the GPU."""
+    """The whole path over every layer of one prefill, inputs resident on the GPU.
+    With a process group the heads are split over its ranks (this rank's slice
+    of every layer's Q/K/V); otherwise this GPU holds all heads."""
 
-    def __init__(self, cfg, lt, device="cuda"):
+    def __init__(self, cfg, lt, device="cuda", group=None):
         self.cfg, self.lt = cfg, lt
-        self.layers = [synth.layer_inputs(cfg, l, device) for l in range(cfg.layers)]
-        T, H, d = cfg.total_tokens, cfg.hq, cfg.d
-        self.cu = torch.tensor(cfg.cu_seqlens(), dtype=torch.int32, device=device) if cfg.batch > 1 else None
-        self.O = torch.empty((T, H, d), dtype=torch.bfloat16, device=device)
-        self.LSE = torch.empty((H, T), dtype=torch.float32, device=device)
-        self.ratio = torch.empty((cfg.layers, cfg.batch, H), dtype=torch.float32, device=device)
-        slots = cfg.S + cfg.W
-        self.K_pool = torch.zeros((cfg.budget, cfg.batch, cfg.hkv, slots, d), dtype=torch.bfloat16, device=device)
-        self.V_pool = torch.zeros_like(self.K_pool)
-        self.pool_len = torch.zeros((cfg.budget, cfg.batch), dtype=torch.int32, device=device)
-        self.Kp = lt.layer_pointer_table([lay[1] for lay in self.layers])
-        self.Vp = lt.layer_pointer_table([lay[2] for lay in self.layers])
-        self.dq = lt.DeviceQueue(cfg.layers, cfg.budget, cfg.batch)
-        self.kw = dict(cu_seqlens=self.cu, max_seqlen=cfg.max_seqlen)
+        if group is not None:
+            q0, q1, k0, k1 = lt.head_shard(cfg.hq, cfg.hkv, torch.distributed.get_rank(group),
+                                           torch.distributed.get_world_size(group))
+        else:
+            q0, q1, k0, k1 = 0, cfg.hq, 0, cfg.hkv
+        layers = []
+        for l in range(cfg.layers):
+            Q, K, V = synth.layer_inputs(cfg, l, device)
+            if group is not None:
+                Q, K, V = Q[:, q0:q1].contiguous(), K[:, k0:k1].contiguous(), V[:, k0:k1].contiguous()
+            layers.append((Q, K, V))
+        self.heads = (q0, q1, k0, k1)
+        self.local = dataclasses.replace(cfg, hq=q1 - q0, hkv=k1 - k0)   # this rank's shape
+        cu = torch.tensor(cfg.cu_seqlens(), dtype=torch.int32, device=device) if cfg.batch > 1 else None
+        self.step = lt.PrefillStep(layers, cfg.budget, cfg.S, cfg.W, cfg.n_obs, cu_seqlens=cu,
+                                   max_seqlen=cfg.max_seqlen, group=group)
+        st = self.step
+        self.layers, self.O, self.LSE, self.ratio = st.layers, st.O, st.LSE, st.ratio
+        self.K_pool, self.V_pool, self.pool_len = st.K_pool, st.V_pool, st.pool_len
+        self.Kp, self.Vp, self.dq, self.kw = st.Kp, st.Vp, st.dq, st.kw
 
-    def enqueue_step(self, stream, events=None, layers=None):
+    def enqueue_step(self, stream, events=None):
         """Enqueue one whole step on `stream`; `events` collects an (start, end)
         pair of external timing events around every attention launch."""
-        cfg, lt = self.cfg, self.lt
-        layers = self.layers if layers is None else layers
-        lt.lt_dqueue_init(self.dq.state, cfg.layers, cfg.budget, cfg.batch, stream)
-        self.ratio.zero_()   # all layers' ratio accumulators, once per step
-        for l in range(cfg.layers):
-            Q, K, V = layers[l]
-            if events is not None:
-                e0 = torch.cuda.Event(enable_timing=True, external=True)
-                e1 = torch.cuda.Event(enable_timing=True, external=True)
-                e0.record(stream)
-            lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, out=self.O, lse=self.LSE, ratio=self.ratio[l],
-                                     stream=stream, accumulate=True, **self.kw)
-            if events is not None:
-                e1.record(stream)
-                events.append((e0, e1))
-            lt.lt_dqueue_push(self.dq.state, cfg.layers, cfg.batch, l, self.ratio[l], stream)
-            lt.lt_compact_kv_pending(self.Kp, self.Vp, self.dq, cfg.S, cfg.W, self.K_pool, self.V_pool,
-                                     self.pool_len, cfg.total_tokens, cfg.hkv, cfg.d, stream=stream, **self.kw)
-
-    @staticmethod
-    def launches_per_step(cfg):
-        # queue init, then attention, push, compaction per layer (the ratio
-        # zeroing once per step is a torch fill)
-        return 1 + 3 * cfg.layers
+        self.step.enqueue(stream, events=events)
 
 
 def run_ours(args, cfg, rank, world):
     import kv_cache_compression_tcgen05_b200 as lt
     lt.library()
     peaks, peak_src = load_peaks()
-    pf = Prefill(cfg, lt)
+    sharded = args.shard == "heads"
+    pf = Prefill(cfg, lt, group=torch.distributed.group.WORLD if sharded else None)
+    lc = pf.local   # this rank's shape: all heads, or its head slice when sharded
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
         pf.enqueue_step(stream)           # eager warm-up: per-device set-up happens outside capture
@@ -249,7 +248,7 @@ def run_ours(args, cfg, rank, world):
     if args.decode_only:
         # One prefill step for the demotions, then the decode leg alone (a
         # short command for profiling the decode kernel).
-        return {"metric": "decode after prefill", "config": cfg.name, **measure_decode(cfg, lt, pf, peaks)}
+        return {"metric": "decode after prefill", "config": cfg.name, **measure_decode(lc, lt, pf, peaks)}
     g_step = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step, stream=stream):
         pf.enqueue_step(stream)
@@ -281,21 +280,29 @@ def run_ours(args, cfg, rank, world):
             stop.record(stream)
         torch.cuda.synchronize()
     barrier(world)
-    launches = args.steps * Prefill.launches_per_step(cfg)
+    launches = args.steps * pf.step.kernel_launches()
     ms = max_over_ranks(start.elapsed_time(stop), world) / args.steps
     with torch.cuda.stream(stream):
         g_events.replay()
     torch.cuda.synchronize()
+    del g_step, g_timed, g_events   # before any process-group teardown (they may hold NCCL calls)
     t_fused = statistics.mean(a.elapsed_time(b) for a, b in fused_ev) * 1e-3
-    # The demotions of the timed steps equal the host queue's on the same ratios.
+    # The demotions of the timed steps equal the host queue's on the same ratios
+    # (all heads' ratios: the gathered ones when the heads are split), and every
+    # rank demotes the same layers.
     mask_dev, order_dev = pf.dq.result()
     host_order = []
+    r = pf.step.all_head_ratios().cpu().numpy()
     for b in range(cfg.batch):
         q = lt.LayerQueue(cfg.layers, cfg.budget)
-        r = pf.ratio.cpu().numpy()
         host_order.append([x for x in (q.push(l, lt.lt_layer_score(r[l, b])) for l in range(cfg.layers)) if x >= 0])
         q.close()
     queue_agrees = all(order_dev[b].tolist() == host_order[b] for b in range(cfg.batch))
+    ranks_agree = True
+    if world > 1:
+        orders = [torch.empty_like(order_dev) for _ in range(world)]
+        torch.distributed.all_gather(orders, order_dev.contiguous())
+        ranks_agree = all(torch.equal(o, orders[0]) for o in orders)
 
     # Beside the step: the plain attention and the separate ratio pass per layer.
     kw = pf.kw
@@ -331,7 +338,7 @@ def run_ours(args, cfg, rank, world):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             Q, K, V = pf.layers[l]
             e0.record()
-            lt.lt_compact_kv(K, V, mask1, cfg.S, cfg.W, k_stream=pf.K_pool[0], v_stream=pf.V_pool[0],
+            lt.lt_compact_kv(K, V, mask1, lc.S, lc.W, k_stream=pf.K_pool[0], v_stream=pf.V_pool[0],
                              stream_len=pf.pool_len[0], **kw)
             e1.record()
             torch.cuda.synchronize()
@@ -346,8 +353,8 @@ def run_ours(args, cfg, rank, world):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        lt.lt_compact_kv_layers(pf.Kp, pf.Vp, demoted_layers, cfg.S, cfg.W, pf.K_pool, pf.V_pool, pf.pool_len,
-                                cfg.total_tokens, cfg.hkv, cfg.d, **kw)
+        lt.lt_compact_kv_layers(pf.Kp, pf.Vp, demoted_layers, lc.S, lc.W, pf.K_pool, pf.V_pool, pf.pool_len,
+                                lc.total_tokens, lc.hkv, lc.d, **kw)
         e1.record()
         torch.cuda.synchronize()
         if rep > 0:
@@ -356,17 +363,19 @@ def run_ours(args, cfg, rank, world):
     t_comp = statistics.mean(c_times)
     t_comp_batch = statistics.median(cb_times)
 
-    fl_attn, fl_ratio = attention_flops(cfg), ratio_flops(cfg)
-    step_flops = cfg.layers * (fl_attn + fl_ratio)
+    # Per-kernel figures are this rank's; the job did world x this rank's work
+    # (replicas: world whole prefills; heads split: one prefill).
+    fl_attn, fl_ratio = attention_flops(lc), ratio_flops(lc)
+    step_flops = lc.layers * (fl_attn + fl_ratio)
     value = world * step_flops / (ms * 1e-3) / 1e12
     achieved = fl_attn / t_fused / 1e12
     peak_sus = float(peaks["bf16_tflops_sustained"])
     peak_burst = float(peaks["bf16_tflops"])
-    traffic = recorded_traffic(cfg.name)
-    comp_gbs = compaction_bytes(cfg, 1) / t_comp / 1e9
+    traffic = recorded_traffic(cfg.name) if lc == cfg else None   # the record is of the all-heads launch
+    comp_gbs = compaction_bytes(lc, 1) / t_comp / 1e9
 
-    decode = measure_decode(cfg, lt, pf, peaks)
-    e2e = measure_e2e(args, cfg, lt, pf, world)
+    decode = measure_decode(lc, lt, pf, peaks)
+    e2e = measure_e2e(args, lc, lt, pf, world)
     cpu = cpu_baseline(cfg) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     clocks = clk.summary()
     line = {
@@ -378,7 +387,7 @@ def run_ours(args, cfg, rank, world):
         "warmup": args.warmup,
         "ms_per_step": round(ms, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V with per-layer sink bias; pages' datasets/weights absent)",
@@ -391,7 +400,9 @@ def run_ours(args, cfg, rank, world):
             "l2": "inputs of one step (all layers' Q/K/V) exceed L2; no flush between steps",
             "step": "one CUDA graph: queue init, all layers' ratio accumulators zeroed once, then per layer fused "
                     "attention+ratio, device queue push, device-driven compaction (programmatic dependent launch)",
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "parallelism": (f"heads split over {world} rank(s): this rank's q heads {pf.heads[0]}..{pf.heads[1] - 1}, "
+                            f"KV heads {pf.heads[2]}..{pf.heads[3] - 1}; ratios all-gathered per layer (NCCL)"
+                            if sharded else f"replicas x{world}" if world > 1 else "single GPU"),
         },
         "attn_tflops": round(achieved, 2),
         "attn_pct_of_burst_peak": round(100 * achieved / peak_burst, 2),
@@ -404,9 +415,10 @@ def run_ours(args, cfg, rank, world):
         "compaction_gbs": round(comp_gbs, 1),
         "compaction_us_per_layer": round(t_comp * 1e6, 2),
         "compaction_batched_layers": n_dem,
-        "compaction_batched_gbs": round(compaction_bytes(cfg, n_dem) / t_comp_batch / 1e9, 1),
-        "separate_ratio_unique_gbs": round(ratio_unique_bytes(cfg) / t_ratio / 1e9, 1),
+        "compaction_batched_gbs": round(compaction_bytes(lc, n_dem) / t_comp_batch / 1e9, 1),
+        "separate_ratio_unique_gbs": round(ratio_unique_bytes(lc) / t_ratio / 1e9, 1),
         "device_queue_matches_host_queue": queue_agrees,
+        "ranks_demote_same_layers": ranks_agree,
         **decode,
         "roofline": {"kernel": "attn_fwd64_kernel (head_dim 64, fused with the lazy ratio)", "bound": "tensor",
                      "achieved": round(achieved, 2), "peak": peak_sus, "unit": "TFLOP/s",
@@ -511,23 +523,23 @@ def measure_e2e(args, cfg, lt, pf, world):
     device-timed region.  Uploads run one layer ahead on a side stream and
     read-backs on another, so copies overlap the kernels; the queue lives on the
     device, so no step waits for the host.  The full K/V of every layer stay on
-    the device (the KV cache the queue manages); Q is double buffered."""
+    the device (the KV cache the queue manages); Q is double buffered.  `cfg` is
+    this rank's shape (its head slice when the heads are split)."""
     host = [tuple(t.cpu().pin_memory() for t in lay) for lay in pf.layers]
     T, H, d = cfg.total_tokens, cfg.hq, cfg.d
     dev_q = [torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     dev_kv = [tuple(torch.empty_like(t) for t in lay[1:]) for lay in pf.layers]
-    Kp = lt.layer_pointer_table([kv[0] for kv in dev_kv])
-    Vp = lt.layer_pointer_table([kv[1] for kv in dev_kv])
+    step = lt.PrefillStep([(dev_q[l % 2],) + dev_kv[l] for l in range(cfg.layers)], cfg.budget, cfg.S, cfg.W,
+                          cfg.n_obs, group=pf.step.group, **pf.kw)
     o_host = torch.empty((cfg.layers, T, H, d), dtype=torch.bfloat16, pin_memory=True)
     lse_host = torch.empty((cfg.layers, H, T), dtype=torch.float32, pin_memory=True)
-    ratio_host = torch.empty(pf.ratio.shape, dtype=torch.float32, pin_memory=True)
-    ks_host = torch.empty(pf.K_pool.shape, dtype=torch.bfloat16, pin_memory=True)
+    ratio_host = torch.empty(step.ratio.shape, dtype=torch.float32, pin_memory=True)
+    ks_host = torch.empty(step.K_pool.shape, dtype=torch.bfloat16, pin_memory=True)
     vs_host = torch.empty_like(ks_host)
     O = [torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     LSE = [torch.empty((H, T), dtype=torch.float32, device="cuda") for _ in range(2)]
     copy_in, copy_out = torch.cuda.Stream(), torch.cuda.Stream()
     main = torch.cuda.current_stream()
-    kw = pf.kw
     h2d = sum(t.numel() * t.element_size() for lay in host for t in lay)
     d2h = o_host.numel() * 2 + lse_host.numel() * 4 + ratio_host.numel() * 4 + 2 * ks_host.numel() * 2
 
@@ -545,18 +557,13 @@ def measure_e2e(args, cfg, lt, pf, world):
                 dev_kv[l][1].copy_(host[l][2], non_blocking=True)
                 ready[l].record(copy_in)
 
-        lt.lt_dqueue_init(pf.dq.state, cfg.layers, cfg.budget, cfg.batch)
+        step.begin(main)
         upload(0)
         for l in range(cfg.layers):
             if l + 1 < cfg.layers:
                 upload(l + 1)
             main.wait_event(ready[l])
-            Q, (K, V) = dev_q[l % 2], dev_kv[l]
-            lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, out=O[l % 2], lse=LSE[l % 2],
-                                     ratio=pf.ratio[l], **kw)
-            lt.lt_dqueue_push(pf.dq.state, cfg.layers, cfg.batch, l, pf.ratio[l])
-            lt.lt_compact_kv_pending(Kp, Vp, pf.dq, cfg.S, cfg.W, pf.K_pool, pf.V_pool, pf.pool_len, T, cfg.hkv, d,
-                                     **kw)
+            step.layer(l, main, O=O[l % 2], LSE=LSE[l % 2])
             computed[l].record(main)
             with torch.cuda.stream(copy_out):
                 copy_out.wait_event(computed[l])
@@ -565,9 +572,9 @@ def measure_e2e(args, cfg, lt, pf, world):
                 done[l].record(copy_out)
         with torch.cuda.stream(copy_out):
             copy_out.wait_stream(main)
-            ratio_host.copy_(pf.ratio, non_blocking=True)
-            ks_host.copy_(pf.K_pool, non_blocking=True)
-            vs_host.copy_(pf.V_pool, non_blocking=True)
+            ratio_host.copy_(step.ratio, non_blocking=True)
+            ks_host.copy_(step.K_pool, non_blocking=True)
+            vs_host.copy_(step.V_pool, non_blocking=True)
         main.wait_stream(copy_out)
         main.wait_stream(copy_in)
 
@@ -657,6 +664,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-only", action="store_true",
                     help="one prefill step, then only the decode measurement (for profiling the decode kernel)")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="with several GPUs: independent replicas (weak scaling, default) or one prefill with its "
+                         "KV heads split over the ranks and the ratios all-gathered per layer (strong scaling)")
     ap.add_argument("--kernels-only", action="store_true",
                     help="time only the device steps (no e2e, CPU baseline or compaction leg); for profiling")
     args = ap.parse_args()
@@ -669,11 +679,12 @@ def main():
         if line is not None:
             print(json.dumps(line), flush=True)
         return
-    rank, world, _ = dist_setup(args.gpus)
-    line = run_ours(args, cfg, rank, world)
+    rank, world, _ = dist_setup(args.gpus, need_group=args.shard == "heads")
+    line = run_ours(args, cfg, rank, world)   # frees its CUDA graphs (they may hold NCCL calls) on return
+    torch.cuda.synchronize()
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if torch.distributed.is_initialized():
         torch.distributed.destroy_process_group()
 
 

@@ -231,6 +231,22 @@ lt_status lt_compact_kv_layers(const lt_shape* shape, const void* const* K_layer
 size_t lt_dqueue_state_bytes(int L, int batch);
 lt_status lt_dqueue_init(void* state, int L, int budget, int batch, lt_stream stream);
 lt_status lt_dqueue_push(void* state, int L, int batch, int layer, const float* ratio, int hq, lt_stream stream);
+
+/*
+ * lt_dqueue_push for ratios gathered from head-sharded ranks: ratio is device
+ * fp32 [shards, batch, hq_shard], where shard n holds query heads
+ * [n hq_shard, (n+1) hq_shard) -- the buffer an all-gather of every rank's
+ * [batch, hq_shard] lt_prefill_attn_ratio output fills.  The score of sequence
+ * b is the mean of its shards * hq_shard head ratios, summed in head order, so
+ * it equals bit for bit the score lt_dqueue_push computes from the same ratios
+ * laid out [batch, hq]; every rank that pushes the same gathered buffer makes
+ * the same demotion.  (The pages describe a single GPU; this split of the
+ * heads over GPUs is this library's reading, with one exchange per layer.)
+ * lt_dqueue_push(..., hq) is lt_dqueue_push_gathered(..., 1, hq).  Errors as
+ * lt_dqueue_push; shards < 1 or hq_shard < 1 is LT_ERR_INVALID_ARG.
+ */
+lt_status lt_dqueue_push_gathered(void* state, int L, int batch, int layer, const float* ratio, int shards,
+                                  int hq_shard, lt_stream stream);
 lt_status lt_dqueue_result(const void* state, int L, int batch, int budget, uint8_t* lazy_mask, int32_t* order,
                            lt_stream stream);
 lt_status lt_dqueue_error(const void* state, int* error_bits);

@@ -6,6 +6,8 @@ arguments: it checks tensor dtypes/devices/shapes, allocates outputs with
 PyTorch when the caller passes none, and calls the library on the current CUDA
 stream.  All arithmetic runs in the library's CUDA kernels; if the library is
 missing the calls raise instead of falling back to anything else.
+``PrefillStep`` (sharded.py) enqueues these calls for every layer of a
+prefill, on one GPU or with the heads split over a process group.
 """
 from __future__ import annotations
 
@@ -41,6 +43,7 @@ from .binding import (  # noqa: F401
     lt_dqueue_error,
     lt_dqueue_init,
     lt_dqueue_push,
+    lt_dqueue_push_gathered,
     lt_dqueue_result,
     lt_dqueue_state_bytes,
     lt_stream_append,
@@ -49,3 +52,4 @@ from .binding import (  # noqa: F401
     lt_stream_ring_init,
 )
 from .build import build  # noqa: F401
+from .sharded import PrefillStep, gather_ratios, head_ratios, head_shard  # noqa: F401

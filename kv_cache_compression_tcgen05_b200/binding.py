@@ -59,6 +59,7 @@ _SIGS = {
     "lt_dqueue_state_bytes": (ctypes.c_size_t, [_i, _i]),
     "lt_dqueue_init": (_i, [_vp, _i, _i, _i, _vp]),
     "lt_dqueue_push": (_i, [_vp, _i, _i, _i, _vp, _i, _vp]),
+    "lt_dqueue_push_gathered": (_i, [_vp, _i, _i, _i, _vp, _i, _i, _vp]),
     "lt_dqueue_result": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp]),
     "lt_dqueue_error": (_i, [_vp, ctypes.POINTER(_i)]),
     "lt_compact_kv_pending": (_i, [_shp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
@@ -359,6 +360,18 @@ def lt_dqueue_push(state, L, batch, layer, ratio, stream=None):
                                     int(ratio.shape[1]), _stream_handle(stream)), "lt_dqueue_push")
 
 
+def lt_dqueue_push_gathered(state, L, batch, layer, gathered, stream=None):
+    """Push of ratios gathered from head-sharded ranks: gathered is device fp32
+    [shards, batch, hq_shard], shard n holding heads [n hq_shard, (n+1) hq_shard)."""
+    _dev_tensor(state, "state", torch.uint8, 1)
+    _dev_tensor(gathered, "gathered", torch.float32, 3)
+    if gathered.shape[1] != batch:
+        raise ValueError("gathered must be [shards, batch, hq_shard]")
+    _check(library().lt_dqueue_push_gathered(state.data_ptr(), int(L), int(batch), int(layer), gathered.data_ptr(),
+                                             int(gathered.shape[0]), int(gathered.shape[2]), _stream_handle(stream)),
+           "lt_dqueue_push_gathered")
+
+
 def lt_dqueue_result(state, L, batch, budget, lazy_mask=None, order=None, stream=None):
     _dev_tensor(state, "state", torch.uint8, 1)
     if lazy_mask is None:
@@ -389,6 +402,9 @@ class DeviceQueue:
 
     def push(self, layer, ratio, stream=None):
         lt_dqueue_push(self.state, self.L, self.batch, layer, ratio, stream)
+
+    def push_gathered(self, layer, gathered, stream=None):
+        lt_dqueue_push_gathered(self.state, self.L, self.batch, layer, gathered, stream)
 
     def result(self, stream=None):
         return lt_dqueue_result(self.state, self.L, self.batch, self.budget, stream=stream)

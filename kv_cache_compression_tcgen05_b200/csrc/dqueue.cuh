@@ -79,10 +79,14 @@ __global__ void dqueue_init_kernel(void* state, int L, int budget, int batch) {
 // Higher score first; on a tie the lower layer index.
 __device__ __forceinline__ bool dq_outranks(float sa, int a, float sb, int b) { return sa != sb ? sa > sb : a < b; }
 
-// One thread per sequence: score = mean of the layer's hq head ratios (summed
-// in double, as the host lt_layer_score does), push, pop the best-ranked
-// layer while more than C = L - budget are queued.
-__global__ void dqueue_push_kernel(void* state, int L, int batch, int layer, const float* ratio, int hq) {
+// One thread per sequence: score = mean of the layer's head ratios (summed in
+// double in head order, as the host lt_layer_score does), push, pop the
+// best-ranked layer while more than C = L - budget are queued.  ratio is
+// [shards, batch, hq_shard]: shard n holds heads [n hq_shard, (n+1) hq_shard)
+// (the all-gather of head-sharded ratios; shards = 1 is the plain [batch, hq]),
+// so the sum runs over the heads in the same order either way.
+__global__ void dqueue_push_kernel(void* state, int L, int batch, int layer, const float* ratio, int hq_shard,
+                                   int shards) {
   pdl_wait();
   pdl_launch_dependents();
   DQueueView v = dqueue_view(state, L, batch);
@@ -94,8 +98,9 @@ __global__ void dqueue_push_kernel(void* state, int L, int batch, int layer, con
   }
   v.last[b] = -1;
   double sum = 0.0;
-  for (int h = 0; h < hq; ++h) sum += ratio[size_t(b) * hq + h];
-  const float score = float(sum / hq);
+  for (int n = 0; n < shards; ++n)
+    for (int h = 0; h < hq_shard; ++h) sum += ratio[(size_t(n) * batch + b) * hq_shard + h];
+  const float score = float(sum / (double(hq_shard) * shards));
   int32_t* pushed = v.pushed + size_t(b) * L;
   if (layer < 0 || layer >= L || pushed[layer] || !isfinite(score)) {
     atomicOr(&v.header[3], kDqErrBadPush);

@@ -402,11 +402,17 @@ lt_status lt_dqueue_init(void* state, int L, int budget, int batch, lt_stream st
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
 }
 
-lt_status lt_dqueue_push(void* state, int L, int batch, int layer, const float* ratio, int hq, lt_stream stream) {
-  if (!dq_args(state, L, batch) || !aligned(ratio, 4) || hq < 1) return LT_ERR_INVALID_ARG;
+lt_status lt_dqueue_push_gathered(void* state, int L, int batch, int layer, const float* ratio, int shards,
+                                  int hq_shard, lt_stream stream) {
+  if (!dq_args(state, L, batch) || !aligned(ratio, 4) || shards < 1 || hq_shard < 1) return LT_ERR_INVALID_ARG;
   const cudaError_t e = launch_pdl(lt::dqueue_push_kernel, dim3(dq_blocks(batch)), dim3(128), 0,
-                                   reinterpret_cast<cudaStream_t>(stream), state, L, batch, layer, ratio, hq);
+                                   reinterpret_cast<cudaStream_t>(stream), state, L, batch, layer, ratio, hq_shard,
+                                   shards);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_dqueue_push(void* state, int L, int batch, int layer, const float* ratio, int hq, lt_stream stream) {
+  return lt_dqueue_push_gathered(state, L, batch, layer, ratio, 1, hq, stream);
 }
 
 lt_status lt_dqueue_result(const void* state, int L, int batch, int budget, uint8_t* lazy_mask, int32_t* order,

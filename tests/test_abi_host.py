@@ -194,6 +194,11 @@ def test_queue_and_pool_calls_reject_bad_arguments():
     assert lib.lt_dqueue_init(FAKE + 4, 4, 2, 1, None) == INV       # state not 16-byte aligned
     assert lib.lt_dqueue_push(FAKE, 0, 1, 0, FAKE, 2, None) == INV   # L < 1
     assert lib.lt_dqueue_push(FAKE, 4, 1, 0, FAKE, 0, None) == INV   # hq < 1
+    # (state, L, batch, layer, ratio, shards, hq_shard)
+    assert lib.lt_dqueue_push_gathered(FAKE, 4, 1, 0, FAKE, 0, 4, None) == INV   # shards < 1
+    assert lib.lt_dqueue_push_gathered(FAKE, 4, 1, 0, FAKE, 2, 0, None) == INV   # hq_shard < 1
+    assert lib.lt_dqueue_push_gathered(FAKE, 4, 0, 0, FAKE, 2, 4, None) == INV   # batch < 1
+    assert lib.lt_dqueue_push_gathered(FAKE, 4, 1, 0, FAKE + 2, 2, 4, None) == INV   # ratio not 4-byte aligned
     # (shape, K_layers, V_layers, state, L, budget, S, W, K_pool, V_pool, pool_len)
     assert lib.lt_compact_kv_pending(ctypes.byref(s), FAKE, FAKE, FAKE, 4, 0, 4, 8, FAKE, FAKE, FAKE, None) == INV
     assert lib.lt_compact_kv_pending(ctypes.byref(s), FAKE, FAKE, FAKE, 4, 2, 0, 0, FAKE, FAKE, FAKE, None) == INV

@@ -1,0 +1,173 @@
+"""The package's prefill step (PrefillStep) and its head-split path, on one GPU.
+
+- lt_dqueue_push_gathered on ratios laid out [shards, batch, hq_shard] makes
+  exactly the pushes lt_dqueue_push makes on the same ratios as [batch, hq];
+- PrefillStep over all heads matches the oracle (ratios, demotions, streaming
+  KV);
+- head slices run one after another on one GPU (no collective: the gathered
+  buffer is assembled by the test), each pushing the gathered ratios of all
+  slices into its own queue, demote the layers the all-heads step demotes and
+  compact exactly their own heads of them, with bit-identical O and LSE;
+- the step with a one-rank NCCL process group (so the ratios take the
+  collective path) captured in a CUDA graph agrees with the step without one.
+"""
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_compression_tcgen05_b200 as lt
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_ready():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    lt.library()
+    yield
+    assert lt.lt_device_status(True) == lt.LT_OK
+
+
+def _cfg():
+    # 600 tokens: several 128-row tiles and a ragged tail; sink-biased layers 1, 3, 4
+    return synth.custom(name="shard", layers=6, seqlens=(600,), hq=8, hkv=4, d=64, S=4, W=64, n_obs=32, budget=3,
+                        seed=11, lazy_layers=(1, 3, 4))
+
+
+def _layers(cfg, q0=0, q1=None, k0=0, k1=None):
+    out = []
+    for l in range(cfg.layers):
+        Q, K, V = synth.layer_inputs(cfg, l, "cuda")
+        out.append((Q[:, q0:q1].contiguous(), K[:, k0:k1].contiguous(), V[:, k0:k1].contiguous()))
+    return out
+
+
+def _step(cfg, layers, group=None):
+    return lt.PrefillStep(layers, cfg.budget, cfg.S, cfg.W, cfg.n_obs, group=group)
+
+
+def _run(step):
+    s = torch.cuda.Stream()
+    step.enqueue(s)
+    torch.cuda.synchronize()
+    assert step.dq.error() == 0
+    _, order = step.dq.result()
+    torch.cuda.synchronize()
+    return order
+
+
+@pytest.mark.parametrize("shards", [1, 2, 4, 8])
+def test_push_gathered_equals_push(shards):
+    L, B, H, budget = 8, 3, 32, 4
+    g = torch.Generator(device="cuda").manual_seed(shards)
+    ratios = torch.rand((L, B, H), generator=g, device="cuda")
+    ratios[5] = ratios[2]                                   # tied layer scores
+    hs = H // shards
+    gathered = ratios.view(L, B, shards, hs).permute(0, 2, 1, 3).contiguous()   # [L, shards, B, hs]
+    a, b = lt.DeviceQueue(L, budget, B), lt.DeviceQueue(L, budget, B)
+    for l in range(L):
+        a.push(l, ratios[l])
+        b.push_gathered(l, gathered[l])
+    ma, oa = a.result()
+    mb, ob = b.result()
+    torch.cuda.synchronize()
+    assert a.error() == 0 and b.error() == 0
+    assert torch.equal(oa, ob) and torch.equal(ma, mb)
+
+
+def test_prefill_step_matches_oracle():
+    cfg = _cfg()
+    layers = _layers(cfg)
+    step = _step(cfg, layers)
+    order = _run(step)[0].tolist()
+    cu = np.array(cfg.cu_seqlens(), np.int32)
+    ref = [oracle.lazy_ratio(cu, synth.bf16_bits(Q), synth.bf16_bits(K), cfg.S, cfg.W, cfg.n_obs)
+           for Q, K, _ in layers]
+    assert np.abs(step.ratio.cpu().numpy() - np.stack(ref)).max() <= 2e-3
+    scores = np.array([r[0].mean() for r in ref])
+    assert order == oracle.queue_online(scores, cfg.budget).tolist()
+    assert sorted(order) == [1, 3, 4]
+    for k, m in enumerate(order):
+        oks, ovs, oln = oracle.compact_kv(cu, synth.bf16_bits(layers[m][1]), synth.bf16_bits(layers[m][2]),
+                                          np.ones(1, np.uint8), cfg.S, cfg.W)
+        assert np.array_equal(synth.bf16_bits(step.K_pool[k, 0]), oks[0])
+        assert np.array_equal(synth.bf16_bits(step.V_pool[k, 0]), ovs[0])
+        assert int(step.pool_len[k, 0]) == int(oln[0])
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_head_slices_on_one_gpu_match_all_heads(world):
+    cfg = _cfg()
+    full = _step(cfg, _layers(cfg))
+    order_full = _run(full)
+    shards = [lt.head_shard(cfg.hq, cfg.hkv, r, world) for r in range(world)]
+    steps = [_step(cfg, _layers(cfg, *sh)) for sh in shards]
+    s = torch.cuda.Stream()
+    for st in steps:                        # each slice's attention + ratios (its own queue is not used)
+        st.enqueue(s)
+    torch.cuda.synchronize()
+    gathered = torch.stack([st.ratio for st in steps], dim=1).contiguous()    # [L, world, B, hq_shard]
+    assert torch.equal(lt.head_ratios(gathered), full.ratio)
+    for (q0, q1, k0, k1), st in zip(shards, steps):
+        assert torch.equal(st.O, full.O[:, q0:q1]) and torch.equal(st.LSE, full.LSE[q0:q1])   # the last layer's
+        # the slice's queue fed every slice's ratios, as after an all-gather
+        with torch.cuda.stream(s):
+            st.K_pool.zero_()
+            st.V_pool.zero_()
+        lt.lt_dqueue_init(st.dq.state, st.L, st.budget, st.batch, s)
+        for l in range(st.L):
+            lt.lt_dqueue_push_gathered(st.dq.state, st.L, st.batch, l, gathered[l], s)
+            lt.lt_compact_kv_pending(st.Kp, st.Vp, st.dq, st.S, st.W, st.K_pool, st.V_pool, st.pool_len, st.T,
+                                     st.hkv, st.d, stream=s)
+        torch.cuda.synchronize()
+        _, order = st.dq.result()
+        torch.cuda.synchronize()
+        assert torch.equal(order, order_full)
+        assert torch.equal(st.K_pool, full.K_pool[:, :, k0:k1]) and torch.equal(st.V_pool, full.V_pool[:, :, k0:k1])
+        assert torch.equal(st.pool_len, full.pool_len)
+
+
+def _free_port():
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        return sock.getsockname()[1]
+
+
+def test_step_with_single_rank_group_in_a_graph():
+    cfg = _cfg()
+    layers = _layers(cfg)
+    plain = _step(cfg, layers)
+    order_plain = _run(plain)
+    dist = torch.distributed
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1)
+    graph = None
+    try:
+        step = _step(cfg, layers, group=dist.group.WORLD)
+        assert step.gathered is not None
+        s = torch.cuda.Stream()
+        with torch.cuda.stream(s):
+            step.enqueue(s)                 # eager: communicator set-up outside capture
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            step.enqueue(s)
+        step.K_pool.zero_()
+        step.ratio.fill_(-1.0)
+        step.gathered.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert step.dq.error() == 0
+        _, order = step.dq.result()
+        torch.cuda.synchronize()
+        assert torch.equal(order, order_plain)
+        assert torch.equal(step.gathered[:, 0], plain.ratio) and torch.equal(step.ratio, plain.ratio)
+        assert torch.equal(step.K_pool, plain.K_pool) and torch.equal(step.V_pool, plain.V_pool)
+    finally:
+        graph = None                        # a graph holding NCCL calls goes before the process group
+        torch.cuda.synchronize()
+        dist.destroy_process_group()
