@@ -205,24 +205,30 @@ class Prefill:
     With a process group the heads are split over its ranks (this rank's slice
     of every layer's Q/K/V); otherwise this GPU holds all heads."""
 
-    def __init__(self, cfg, lt, device="cuda", group=None):
+    def __init__(self, cfg, lt, device="cuda", group=None, seqs=None):
         self.cfg, self.lt = cfg, lt
         if group is not None:
             q0, q1, k0, k1 = lt.head_shard(cfg.hq, cfg.hkv, torch.distributed.get_rank(group),
                                            torch.distributed.get_world_size(group))
         else:
             q0, q1, k0, k1 = 0, cfg.hq, 0, cfg.hkv
+        self.seqs = list(range(cfg.batch)) if seqs is None else list(seqs)
         layers = []
         for l in range(cfg.layers):
             Q, K, V = synth.layer_inputs(cfg, l, device)
             if group is not None:
                 Q, K, V = Q[:, q0:q1].contiguous(), K[:, k0:k1].contiguous(), V[:, k0:k1].contiguous()
+            if seqs is not None:
+                Q, K, V = (lt.pack_sequences(t, cfg.cu_seqlens(), self.seqs)[0] for t in (Q, K, V))
             layers.append((Q, K, V))
         self.heads = (q0, q1, k0, k1)
-        self.local = dataclasses.replace(cfg, hq=q1 - q0, hkv=k1 - k0)   # this rank's shape
-        cu = torch.tensor(cfg.cu_seqlens(), dtype=torch.int32, device=device) if cfg.batch > 1 else None
+        # this rank's shape: its heads and its sequences
+        self.local = dataclasses.replace(cfg, hq=q1 - q0, hkv=k1 - k0,
+                                         seqlens=tuple(cfg.seqlens[b] for b in self.seqs))
+        lc = self.local
+        cu = torch.tensor(lc.cu_seqlens(), dtype=torch.int32, device=device) if lc.batch > 1 else None
         self.step = lt.PrefillStep(layers, cfg.budget, cfg.S, cfg.W, cfg.n_obs, cu_seqlens=cu,
-                                   max_seqlen=cfg.max_seqlen, group=group)
+                                   max_seqlen=lc.max_seqlen, group=group)
         st = self.step
         self.layers, self.O, self.LSE, self.ratio = st.layers, st.O, st.LSE, st.ratio
         self.K_pool, self.V_pool, self.pool_len = st.K_pool, st.V_pool, st.pool_len
@@ -238,10 +244,12 @@ def run_ours(args, cfg, rank, world):
     import kv_cache_compression_tcgen05_b200 as lt
     lt.library()
     peaks, peak_src = load_peaks()
-    sharded = args.shard == "heads"
-    pf = Prefill(cfg, lt, group=torch.distributed.group.WORLD if sharded else None)
-    lc = pf.local   # this rank's shape: all heads, or its head slice when sharded
+    sharded = args.shard != "replicas"
+    pf = Prefill(cfg, lt, group=torch.distributed.group.WORLD if args.shard == "heads" else None,
+                 seqs=lt.sequence_shard(cfg.seqlens, rank, world) if args.shard == "sequences" else None)
+    lc = pf.local   # this rank's shape: all heads and sequences, or its slice when sharded
     stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())   # the inputs were made on the default stream
     with torch.cuda.stream(stream):
         pf.enqueue_step(stream)           # eager warm-up: per-device set-up happens outside capture
     torch.cuda.synchronize()
@@ -293,13 +301,13 @@ def run_ours(args, cfg, rank, world):
     mask_dev, order_dev = pf.dq.result()
     host_order = []
     r = pf.step.all_head_ratios().cpu().numpy()
-    for b in range(cfg.batch):
+    for b in range(lc.batch):
         q = lt.LayerQueue(cfg.layers, cfg.budget)
         host_order.append([x for x in (q.push(l, lt.lt_layer_score(r[l, b])) for l in range(cfg.layers)) if x >= 0])
         q.close()
-    queue_agrees = all(order_dev[b].tolist() == host_order[b] for b in range(cfg.batch))
+    queue_agrees = all(order_dev[b].tolist() == host_order[b] for b in range(lc.batch))
     ranks_agree = True
-    if world > 1:
+    if world > 1 and args.shard == "heads":
         orders = [torch.empty_like(order_dev) for _ in range(world)]
         torch.distributed.all_gather(orders, order_dev.contiguous())
         ranks_agree = all(torch.equal(o, orders[0]) for o in orders)
@@ -329,7 +337,7 @@ def run_ours(args, cfg, rank, world):
                 "gpu_launches": launches}
 
     # Compaction timed on its own: every demoted layer of one step (inputs > L2 apart).
-    mask1 = torch.ones(cfg.batch, dtype=torch.uint8, device="cuda")
+    mask1 = torch.ones(lc.batch, dtype=torch.uint8, device="cuda")
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device="cuda")
     c_times = []
     for rep in range(5):
@@ -363,11 +371,11 @@ def run_ours(args, cfg, rank, world):
     t_comp = statistics.mean(c_times)
     t_comp_batch = statistics.median(cb_times)
 
-    # Per-kernel figures are this rank's; the job did world x this rank's work
-    # (replicas: world whole prefills; heads split: one prefill).
+    # Per-kernel figures are this rank's; the job is world whole prefills
+    # (replicas) or the one prefill split over the ranks.
     fl_attn, fl_ratio = attention_flops(lc), ratio_flops(lc)
-    step_flops = lc.layers * (fl_attn + fl_ratio)
-    value = world * step_flops / (ms * 1e-3) / 1e12
+    job_flops = cfg.layers * (attention_flops(cfg) + ratio_flops(cfg)) * (1 if sharded else world)
+    value = job_flops / (ms * 1e-3) / 1e12
     achieved = fl_attn / t_fused / 1e12
     peak_sus = float(peaks["bf16_tflops_sustained"])
     peak_burst = float(peaks["bf16_tflops"])
@@ -375,7 +383,7 @@ def run_ours(args, cfg, rank, world):
     comp_gbs = compaction_bytes(lc, 1) / t_comp / 1e9
 
     decode = measure_decode(lc, lt, pf, peaks)
-    e2e = measure_e2e(args, lc, lt, pf, world)
+    e2e = measure_e2e(args, lc, lt, pf, world, job_flops)
     cpu = cpu_baseline(cfg) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     clocks = clk.summary()
     line = {
@@ -402,7 +410,10 @@ def run_ours(args, cfg, rank, world):
                     "attention+ratio, device queue push, device-driven compaction (programmatic dependent launch)",
             "parallelism": (f"heads split over {world} rank(s): this rank's q heads {pf.heads[0]}..{pf.heads[1] - 1}, "
                             f"KV heads {pf.heads[2]}..{pf.heads[3] - 1}; ratios all-gathered per layer (NCCL)"
-                            if sharded else f"replicas x{world}" if world > 1 else "single GPU"),
+                            if args.shard == "heads" else
+                            f"sequences split over {world} rank(s) by causal work: rank 0's sequences {pf.seqs}; "
+                            f"no exchange" if args.shard == "sequences" else
+                            f"replicas x{world}" if world > 1 else "single GPU"),
         },
         "attn_tflops": round(achieved, 2),
         "attn_pct_of_burst_peak": round(100 * achieved / peak_burst, 2),
@@ -516,7 +527,7 @@ def measure_decode(cfg, lt, pf, peaks):
     return out
 
 
-def measure_e2e(args, cfg, lt, pf, world):
+def measure_e2e(args, cfg, lt, pf, world, job_flops):
     """Same metric through the public calls with host buffers: every step copies
     each layer's Q/K/V from pinned host memory to the device and reads back each
     layer's O and LSE, the ratios and the streaming KV pool, all inside the
@@ -524,7 +535,8 @@ def measure_e2e(args, cfg, lt, pf, world):
     read-backs on another, so copies overlap the kernels; the queue lives on the
     device, so no step waits for the host.  The full K/V of every layer stay on
     the device (the KV cache the queue manages); Q is double buffered.  `cfg` is
-    this rank's shape (its head slice when the heads are split)."""
+    this rank's shape (its slice when the heads or sequences are split);
+    job_flops the work of the whole job per step."""
     host = [tuple(t.cpu().pin_memory() for t in lay) for lay in pf.layers]
     T, H, d = cfg.total_tokens, cfg.hq, cfg.d
     dev_q = [torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
@@ -590,8 +602,7 @@ def measure_e2e(args, cfg, lt, pf, world):
     e1.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
-    step_flops = cfg.layers * (attention_flops(cfg) + ratio_flops(cfg))
-    return {"value": round(world * step_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+    return {"value": round(job_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 3)}
 
 
@@ -664,9 +675,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-only", action="store_true",
                     help="one prefill step, then only the decode measurement (for profiling the decode kernel)")
-    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
-                    help="with several GPUs: independent replicas (weak scaling, default) or one prefill with its "
-                         "KV heads split over the ranks and the ratios all-gathered per layer (strong scaling)")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads", "sequences"],
+                    help="with several GPUs: independent replicas (weak scaling, default); one prefill with its "
+                         "KV heads split over the ranks and the ratios all-gathered per layer; or a packed batch "
+                         "split by whole sequences, no exchange (both strong scaling)")
     ap.add_argument("--kernels-only", action="store_true",
                     help="time only the device steps (no e2e, CPU baseline or compaction leg); for profiling")
     args = ap.parse_args()

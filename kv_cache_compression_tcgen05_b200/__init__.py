@@ -52,4 +52,11 @@ from .binding import (  # noqa: F401
     lt_stream_ring_init,
 )
 from .build import build  # noqa: F401
-from .sharded import PrefillStep, gather_ratios, head_ratios, head_shard  # noqa: F401
+from .sharded import (  # noqa: F401
+    PrefillStep,
+    gather_ratios,
+    head_ratios,
+    head_shard,
+    pack_sequences,
+    sequence_shard,
+)

@@ -8,8 +8,12 @@ demotes (LightTransfer project page, Methodology, LightTransfer-Test; the
 LightTransfer write-up, second solution).  No step waits for the host, so the
 whole step can be captured in one CUDA graph.
 
-Head sharding (one process per GPU; the pages describe a single GPU, the split
-is this library's reading): rank r of N holds KV heads [r Hkv/N, (r+1) Hkv/N)
+Sequence sharding of a packed batch (sequence_shard, pack_sequences): each rank
+takes whole sequences and runs its own PrefillStep on them; the sequences'
+queues are independent, so nothing is exchanged.
+
+Head sharding (one process per GPU; the pages describe a single GPU, both
+splits are this library's reading): rank r of N holds KV heads [r Hkv/N, (r+1) Hkv/N)
 and the query heads of their groups -- the contiguous slices a column-sharded
 QKV projection produces -- and runs attention, the ratio and the compaction on
 those heads alone.  The layer score is the mean of the ratios of all Hq query
@@ -40,6 +44,37 @@ def head_shard(hq: int, hkv: int, rank: int, world: int):
     g, per = hq // hkv, hkv // world
     kv0 = rank * per
     return kv0 * g, (kv0 + per) * g, kv0, kv0 + per
+
+
+def sequence_shard(seqlens, rank: int, world: int):
+    """Sequences of `rank` when a packed batch is split over `world` ranks by
+    whole sequences (independent prefills: no exchange, every rank keeps its own
+    sequences' queues).  Sequences are dealt largest causal work N(N+1)/2 first,
+    each to the rank with the least work so far (ties: lower sequence index,
+    lower rank), so the slowest rank stays near 1/world of the batch's work.
+    Returned in increasing order; the same on every rank."""
+    seqlens = [int(n) for n in seqlens]
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("rank must lie in [0, world)")
+    if len(seqlens) < world:
+        raise ValueError(f"{len(seqlens)} sequences cannot feed {world} ranks")
+    load, owner = [0] * world, [0] * len(seqlens)
+    for b in sorted(range(len(seqlens)), key=lambda b: (-seqlens[b] * (seqlens[b] + 1), b)):
+        r = min(range(world), key=lambda r: (load[r], r))
+        owner[b] = r
+        load[r] += seqlens[b] * (seqlens[b] + 1) // 2
+    return [b for b in range(len(seqlens)) if owner[b] == rank]
+
+
+def pack_sequences(t: torch.Tensor, cu_seqlens, seqs):
+    """Rows of the listed sequences of a packed [T, ...] tensor, packed in the
+    listed order, and their cu_seqlens (a list, from 0)."""
+    cu = [int(x) for x in cu_seqlens]
+    parts, local_cu = [], [0]
+    for b in seqs:
+        parts.append(t[cu[b]:cu[b + 1]])
+        local_cu.append(local_cu[-1] + cu[b + 1] - cu[b])
+    return torch.cat(parts, dim=0).contiguous(), local_cu
 
 
 def gather_ratios(ratio_local: torch.Tensor, gathered: torch.Tensor, group=None) -> None:

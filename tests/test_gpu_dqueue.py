@@ -144,6 +144,7 @@ def test_graph_captured_tiny_prefill():
             lt.lt_compact_kv_pending(Kp, Vp, dq, cfg.S, cfg.W, K_pool, V_pool, pool_len, T, cfg.hkv, d, stream=stream)
 
     s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())   # the inputs were made on the default stream
     with torch.cuda.stream(s):
         prefill(s)            # warm-up outside capture (first calls set up per-device state)
     torch.cuda.synchronize()

@@ -9,7 +9,8 @@
   slices into its own queue, demote the layers the all-heads step demotes and
   compact exactly their own heads of them, with bit-identical O and LSE;
 - the step with a one-rank NCCL process group (so the ratios take the
-  collective path) captured in a CUDA graph agrees with the step without one.
+  collective path) captured in a CUDA graph agrees with the step without one;
+- ranks that take whole sequences of a packed batch reproduce the batch's rows.
 """
 import socket
 
@@ -53,6 +54,7 @@ def _step(cfg, layers, group=None):
 
 def _run(step):
     s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())     # inputs and the step's buffers were made there
     step.enqueue(s)
     torch.cuda.synchronize()
     assert step.dq.error() == 0
@@ -108,6 +110,7 @@ def test_head_slices_on_one_gpu_match_all_heads(world):
     shards = [lt.head_shard(cfg.hq, cfg.hkv, r, world) for r in range(world)]
     steps = [_step(cfg, _layers(cfg, *sh)) for sh in shards]
     s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
     for st in steps:                        # each slice's attention + ratios (its own queue is not used)
         st.enqueue(s)
     torch.cuda.synchronize()
@@ -150,6 +153,7 @@ def test_step_with_single_rank_group_in_a_graph():
         step = _step(cfg, layers, group=dist.group.WORLD)
         assert step.gathered is not None
         s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
             step.enqueue(s)                 # eager: communicator set-up outside capture
         torch.cuda.synchronize()
@@ -171,3 +175,33 @@ def test_step_with_single_rank_group_in_a_graph():
         graph = None                        # a graph holding NCCL calls goes before the process group
         torch.cuda.synchronize()
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sequence_slices_match_full_batch(world):
+    """Ranks that take whole sequences of a packed batch (run one after another
+    here) reproduce the full batch's rows: bit-identical O, LSE, demotions and
+    streaming KV per sequence; the ratios agree to float-atomic order (the
+    observed rows of a sequence can span two query tiles)."""
+    cfg = synth.custom(name="seqs", layers=5, seqlens=(300, 77, 520, 190), hq=4, hkv=2, d=64, S=4, W=48, n_obs=24,
+                       budget=2, seed=13, lazy_layers=(1, 3))
+    layers = _layers(cfg)
+    cu_h = cfg.cu_seqlens()
+    full = lt.PrefillStep(layers, cfg.budget, cfg.S, cfg.W, cfg.n_obs,
+                          cu_seqlens=torch.tensor(cu_h, dtype=torch.int32, device="cuda"), max_seqlen=cfg.max_seqlen)
+    order_full = _run(full)
+    for r in range(world):
+        seqs = lt.sequence_shard(cfg.seqlens, r, world)
+        packed = [tuple(lt.pack_sequences(t, cu_h, seqs)[0] for t in lay) for lay in layers]
+        local_cu = lt.pack_sequences(layers[0][0], cu_h, seqs)[1]
+        cu = torch.tensor(local_cu, dtype=torch.int32, device="cuda") if len(seqs) > 1 else None
+        st = lt.PrefillStep(packed, cfg.budget, cfg.S, cfg.W, cfg.n_obs, cu_seqlens=cu,
+                            max_seqlen=max(cfg.seqlens[b] for b in seqs))
+        order = _run(st)
+        for i, b in enumerate(seqs):
+            assert torch.equal(order[i], order_full[b])
+            assert torch.allclose(st.ratio[:, i], full.ratio[:, b], rtol=0, atol=1e-6)
+            assert torch.equal(st.K_pool[:, i], full.K_pool[:, b]) and torch.equal(st.V_pool[:, i], full.V_pool[:, b])
+            assert torch.equal(st.pool_len[:, i], full.pool_len[:, b])
+            l0, l1, g0, g1 = local_cu[i], local_cu[i + 1], cu_h[b], cu_h[b + 1]
+            assert torch.equal(st.O[l0:l1], full.O[g0:g1]) and torch.equal(st.LSE[:, l0:l1], full.LSE[:, g0:g1])

@@ -1,8 +1,10 @@
-"""Head sharding on the CPU: the head ranges, the global head order of gathered
-ratios, and two gloo ranks that each compute their own heads' lazy ratios (with
-the oracle), all-gather them with the library's gather_ratios and run the
-library's host queue on the gathered scores.  Both ranks must demote the same
-layers as one process holding all heads, with bit-identical layer scores."""
+"""Sharding on the CPU.  Heads: the head ranges, the global head order of
+gathered ratios, and two gloo ranks that each compute their own heads' lazy
+ratios (with the oracle), all-gather them with the library's gather_ratios and
+run the library's host queue on the gathered scores; both ranks must demote the
+same layers as one process holding all heads, with bit-identical layer scores.
+Sequences: every sequence dealt to one rank, the slowest rank's work within the
+greedy bound, and packing of a rank's sequences."""
 import os
 import socket
 
@@ -121,3 +123,36 @@ def test_two_gloo_ranks_demote_as_one_process():
     single = _demotions(cfg, lambda layer: _ratios(cfg, layer, 0, cfg.hq, 0, cfg.hkv))
     assert len(single[0]) == cfg.budget
     assert out[0] == out[1] == single     # same demotion order and bit-identical scores
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+def test_sequence_shard_deals_every_sequence_once_and_balances(world):
+    import synth
+    seqlens = synth.CONFIGS["batched"].seqlens
+    parts = [lt.sequence_shard(seqlens, r, world) for r in range(world)]
+    assert sorted(b for p in parts for b in p) == list(range(len(seqlens)))
+    assert all(p == sorted(p) and p for p in parts)
+    work = [n * (n + 1) // 2 for n in seqlens]
+    loads = [sum(work[b] for b in p) for p in parts]
+    # greedy largest-first bound: the slowest rank exceeds the mean by at most one sequence's work
+    assert max(loads) <= sum(work) / world + max(work)
+    assert parts == [lt.sequence_shard(list(seqlens), r, world) for r in range(world)]   # deterministic
+
+
+def test_sequence_shard_examples_and_errors():
+    # works 55, 820, 210, 465: 40 -> r0 (820); 30 -> r1 (465); 20 -> r1 (675); 10 -> r1 (730)
+    assert lt.sequence_shard([10, 40, 20, 30], 0, 2) == [1]
+    assert lt.sequence_shard([10, 40, 20, 30], 1, 2) == [0, 2, 3]
+    assert lt.sequence_shard([5, 5, 5], 2, 3) == [2]
+    with pytest.raises(ValueError):
+        lt.sequence_shard([5, 5], 0, 3)
+    with pytest.raises(ValueError):
+        lt.sequence_shard([5, 5], 2, 2)
+
+
+def test_pack_sequences_keeps_rows_and_lengths():
+    cu = [0, 3, 7, 12]
+    t = torch.arange(12 * 2).reshape(12, 2)
+    packed, local_cu = lt.pack_sequences(t, cu, [2, 0])
+    assert local_cu == [0, 5, 8]
+    assert torch.equal(packed, torch.cat([t[7:12], t[0:3]]))
