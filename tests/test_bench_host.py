@@ -1,0 +1,70 @@
+"""Host logic of bench.py that the reported numbers rest on, checked without a GPU:
+the algorithmic work counts (closed forms against brute-force enumeration of
+the key sets the method defines) and the parsing of the nvidia-smi clock
+samples that decide whether a run is kept."""
+import bench
+import synth
+
+
+def _key_set(i, S, W):
+    """K_i: the sink keys [0, min(S, i+1)) and the window [max(S, i-W+1), i]."""
+    return set(range(min(S, i + 1))) | set(range(max(S, i - W + 1), i + 1))
+
+
+def _cases():
+    yield synth.custom(name="a", seqlens=(37,), hq=4, hkv=2, d=64, S=4, W=8, n_obs=16)
+    yield synth.custom(name="b", seqlens=(3, 50, 9), hq=6, hkv=3, d=128, S=4, W=5, n_obs=12)
+    yield synth.custom(name="c", seqlens=(20,), hq=2, hkv=1, d=64, S=0, W=1, n_obs=30)
+    yield synth.custom(name="d", seqlens=(12,), hq=2, hkv=1, d=64, S=6, W=40, n_obs=5)
+
+
+def test_attention_flops_count_causal_pairs():
+    for cfg in _cases():
+        pairs = sum(1 for n in cfg.seqlens for i in range(n) for j in range(n) if j <= i)
+        assert bench.attention_flops(cfg) == 4 * cfg.d * cfg.hq * pairs
+
+
+def test_ratio_flops_count_the_observed_rows_key_sets():
+    for cfg in _cases():
+        keys = 0
+        for n in cfg.seqlens:
+            for i in range(max(0, n - cfg.n_obs), n):
+                keys += len(_key_set(i, cfg.S, cfg.W))
+        assert bench.ratio_flops(cfg) == 2 * cfg.d * cfg.hq * keys
+
+
+def test_ratio_unique_bytes_count_the_union_of_touched_rows():
+    for cfg in _cases():
+        total = 0
+        for n in cfg.seqlens:
+            obs = range(max(0, n - cfg.n_obs), n)
+            rows = set().union(*(_key_set(i, cfg.S, cfg.W) for i in obs))
+            total += len(obs) * cfg.hq * (2 * cfg.d + 4) + len(rows) * cfg.hkv * 2 * cfg.d
+        assert bench.ratio_unique_bytes(cfg) == total
+
+
+def test_compaction_bytes_count_the_kept_rows():
+    for cfg in _cases():
+        kept = 0
+        for n in cfg.seqlens:
+            p = list(range(min(cfg.S, n))) + list(range(max(cfg.S, n - cfg.W), n))
+            assert len(p) == len(set(p))
+            kept += len(p)
+        # K and V, each read and written, bf16
+        assert bench.compaction_bytes(cfg, 3) == 3 * 2 * 2 * kept * cfg.hkv * cfg.d * 2
+
+
+def test_clock_summary_reads_median_and_throttle_reasons():
+    cs = bench.ClockSampler(0)
+    cs.lines = [
+        "0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1950, 1965, 950.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+        "0, [N/A], 1965, 1.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    s = cs.summary()
+    assert s["sm_mhz"] == 1950.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["sw_power_cap"]
+    cs.lines = ["0, 1500, 1965, 900, 0x8, Active, Not Active, Active, Not Active"]
+    assert cs.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
