@@ -126,6 +126,14 @@ def _dev_tensor(t, name, dtype, ndim=None):
     return t
 
 
+def _sized(t, name, dtype, shape):
+    """A caller's device tensor that must have exactly `shape` (the library indexes it so)."""
+    _dev_tensor(t, name, dtype, len(shape))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
 def _shape(T, hq, hkv, d, cu_seqlens, max_seqlen):
     s = LtShape()
     s.total_tokens = int(T)
@@ -254,7 +262,7 @@ def lt_compact_kv(K, V, mask, S, W, cu_seqlens=None, max_seqlen=None, k_stream=N
         _dev_tensor(t, n, torch.bfloat16, 4)
         if t.shape != (shape.batch, hkv, slots, d):
             raise ValueError(f"{n} must be [batch, hkv, S+W, d]")
-    _dev_tensor(stream_len, "stream_len", torch.int32, 1)
+    _sized(stream_len, "stream_len", torch.int32, (shape.batch,))
     _check(library().lt_compact_kv(ctypes.byref(shape), K.data_ptr(), V.data_ptr(), mask.data_ptr(), int(S),
                                    int(W), k_stream.data_ptr(), v_stream.data_ptr(), stream_len.data_ptr(),
                                    _stream_handle(stream)), "lt_compact_kv")
@@ -378,6 +386,8 @@ def lt_dqueue_result(state, L, batch, budget, lazy_mask=None, order=None, stream
         lazy_mask = torch.empty((batch, L), dtype=torch.uint8, device=state.device)
     if order is None:
         order = torch.empty((batch, max(int(budget), 1)), dtype=torch.int32, device=state.device)
+    _sized(lazy_mask, "lazy_mask", torch.uint8, (batch, L))
+    _sized(order, "order", torch.int32, (batch, max(int(budget), 1)))
     _check(library().lt_dqueue_result(state.data_ptr(), int(L), int(batch), int(budget), lazy_mask.data_ptr(),
                                       order.data_ptr(), _stream_handle(stream)), "lt_dqueue_result")
     return lazy_mask, order[:, : int(budget)]
@@ -431,7 +441,7 @@ def lt_compact_kv_pending(K_layers, V_layers, queue, S, W, K_pool, V_pool, pool_
         _dev_tensor(t, n, torch.bfloat16, 5)
         if t.shape != (queue.budget, queue.batch, hkv, slots, d):
             raise ValueError(f"{n} must be [budget, batch, hkv, S+W, d]")
-    _dev_tensor(pool_len, "pool_len", torch.int32, 2)
+    _sized(pool_len, "pool_len", torch.int32, (queue.budget, queue.batch))
     shape = _shape(total_tokens, hkv, hkv, d, cu_seqlens, max_seqlen)
     if shape.batch != queue.batch:
         raise ValueError("batch differs from the queue's")
@@ -458,7 +468,7 @@ def lt_compact_kv_layers(K_layers, V_layers, layers, S, W, K_pool, V_pool, pool_
         _dev_tensor(t, nm, torch.bfloat16, 5)
         if t.shape != (n, shape.batch, hkv, slots, d):
             raise ValueError(f"{nm} must be [n, batch, hkv, S+W, d]")
-    _dev_tensor(pool_len, "pool_len", torch.int32, 2)
+    _sized(pool_len, "pool_len", torch.int32, (n, shape.batch))
     _check(library().lt_compact_kv_layers(ctypes.byref(shape), K_layers.data_ptr(), V_layers.data_ptr(), L,
                                           layers.data_ptr(), n, int(S), int(W), K_pool.data_ptr(), V_pool.data_ptr(),
                                           pool_len.data_ptr(), _stream_handle(stream)), "lt_compact_kv_layers")
@@ -466,7 +476,7 @@ def lt_compact_kv_layers(K_layers, V_layers, layers, S, W, K_pool, V_pool, pool_
 
 def lt_stream_ring_init(stream_len, next_slot, S, W, stream=None):
     _dev_tensor(stream_len, "stream_len", torch.int32, 1)
-    _dev_tensor(next_slot, "next_slot", torch.int32, 1)
+    _sized(next_slot, "next_slot", torch.int32, (stream_len.numel(),))
     _check(library().lt_stream_ring_init(stream_len.data_ptr(), next_slot.data_ptr(), stream_len.numel(), int(S),
                                          int(W), _stream_handle(stream)), "lt_stream_ring_init")
 
@@ -482,8 +492,8 @@ def lt_stream_append(K_stream, V_stream, stream_len, next_slot, k_new, v_new, S,
         _dev_tensor(t, n, torch.bfloat16, 3)
         if t.shape != (B, hkv, d):
             raise ValueError(f"{n} must be [batch, hkv, d]")
-    _dev_tensor(stream_len, "stream_len", torch.int32, 1)
-    _dev_tensor(next_slot, "next_slot", torch.int32, 1)
+    _sized(stream_len, "stream_len", torch.int32, (B,))
+    _sized(next_slot, "next_slot", torch.int32, (B,))
     _check(library().lt_stream_append(K_stream.data_ptr(), V_stream.data_ptr(), stream_len.data_ptr(),
                                       next_slot.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), B, hkv, d, int(S),
                                       int(W), _stream_handle(stream)), "lt_stream_append")
@@ -498,11 +508,13 @@ def lt_stream_decode(q, K_stream, V_stream, stream_len, softmax_scale=None, out=
     _, hkv, slots, dk = K_stream.shape
     if K_stream.shape[0] != B or dk != d or V_stream.shape != K_stream.shape:
         raise ValueError("caches must be [batch, hkv, S+W, d] with q's batch and d")
-    _dev_tensor(stream_len, "stream_len", torch.int32, 1)
+    _sized(stream_len, "stream_len", torch.int32, (B,))
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    _sized(out, "out", torch.bfloat16, (B, hq, d))
+    _sized(lse, "lse", torch.float32, (B, hq))
     _check(library().lt_stream_decode(q.data_ptr(), K_stream.data_ptr(), V_stream.data_ptr(), stream_len.data_ptr(),
                                       B, hq, hkv, d, slots, out.data_ptr(), lse.data_ptr(),
                                       0.0 if softmax_scale is None else float(softmax_scale), _stream_handle(stream)),
@@ -539,11 +551,15 @@ def lt_decode_attn(q, K, V, seq_len, seq_start=None, max_len=None, softmax_scale
         limit = rows if max_len is None else int(max_len)
     if dk != d or V.shape != K.shape:
         raise ValueError("K and V must have the same shape and q's head dim")
-    _dev_tensor(seq_len, "seq_len", torch.int32, 1)
+    _sized(seq_len, "seq_len", torch.int32, (B,))
+    if seq_start is not None:
+        _sized(seq_start, "seq_start", torch.int32, (B,))
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
+    _sized(out, "out", torch.bfloat16, (B, hq, d))
+    _sized(lse, "lse", torch.float32, (B, hq))
     _check(library().lt_decode_attn(q.data_ptr(), K.data_ptr(), V.data_ptr(),
                                     None if seq_start is None else seq_start.data_ptr(), cap, seq_len.data_ptr(), B,
                                     hq, hkv, d, limit, out.data_ptr(), lse.data_ptr(),

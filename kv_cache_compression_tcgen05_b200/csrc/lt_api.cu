@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <algorithm>
@@ -22,6 +23,18 @@
 #include "lt.h"
 
 namespace {
+
+// One NVTX range per library call, named after the entry point, so that a
+// profiler's timeline and `ncu --nvtx` filters show which call enqueued which
+// kernels.  Host side only (a graph replay runs none of it); with no tool
+// attached each push/pop is a call through a no-op pointer.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
+#define LT_RANGE() const CallRange lt_call_range_(__func__)
 
 // Device status word: bit lt::kErrTimeout is set by a kernel that gave up a
 // bounded wait.  One copy per device; read and cleared by lt_device_status.
@@ -237,12 +250,14 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
 
 lt_status lt_prefill_attn(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O, float* LSE,
                           float softmax_scale, lt_stream stream) {
+  LT_RANGE();
   return launch_attention(shape, Q, K, V, O, LSE, softmax_scale, 0, 0, 0, nullptr, stream);
 }
 
 lt_status lt_prefill_attn_ratio(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
                                 float* LSE, float softmax_scale, int S, int W, int n_obs, float* ratio,
                                 lt_stream stream) {
+  LT_RANGE();
   if (!ratio) return LT_ERR_INVALID_ARG;
   return launch_attention(shape, Q, K, V, O, LSE, softmax_scale, S, W, n_obs, ratio, stream);
 }
@@ -250,12 +265,14 @@ lt_status lt_prefill_attn_ratio(const lt_shape* shape, const void* Q, const void
 lt_status lt_prefill_attn_ratio_acc(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
                                     float* LSE, float softmax_scale, int S, int W, int n_obs, float* ratio,
                                     lt_stream stream) {
+  LT_RANGE();
   if (!ratio) return LT_ERR_INVALID_ARG;
   return launch_attention(shape, Q, K, V, O, LSE, softmax_scale, S, W, n_obs, ratio, stream, false);
 }
 
 lt_status lt_lazy_ratio(const lt_shape* shape, const void* Q, const void* K, const float* LSE, float softmax_scale,
                         int S, int W, int n_obs, float* ratio, lt_stream stream) {
+  LT_RANGE();
   lt_status st = check_shape(shape);
   if (st != LT_OK) return st;
   // With no tokens only `ratio` is written (zeros); the inputs may be null.
@@ -314,6 +331,7 @@ lt_status lt_lazy_ratio(const lt_shape* shape, const void* Q, const void* K, con
 
 lt_status lt_compact_kv(const lt_shape* shape, const void* K, const void* V, const uint8_t* mask, int S, int W,
                         void* K_stream, void* V_stream, int32_t* stream_len, lt_stream stream) {
+  LT_RANGE();
   lt_status st = check_shape(shape);
   if (st != LT_OK) return st;
   if (!mask || !aligned(K_stream, 16) || !aligned(V_stream, 16) || !aligned(stream_len, 4)) return LT_ERR_INVALID_ARG;
@@ -347,6 +365,7 @@ lt_status lt_compact_kv(const lt_shape* shape, const void* K, const void* V, con
 lt_status lt_compact_kv_layers(const lt_shape* shape, const void* const* K_layers, const void* const* V_layers, int L,
                                const int32_t* layers, int n, int S, int W, void* K_pool, void* V_pool,
                                int32_t* pool_len, lt_stream stream) {
+  LT_RANGE();
   lt_status st = check_shape(shape);
   if (st != LT_OK) return st;
   if (L < 1 || n < 0 || n > L || !aligned(K_layers, 8) || !aligned(V_layers, 8) ||
@@ -393,6 +412,7 @@ static bool dq_args(const void* state, int L, int batch) {
 static int dq_blocks(int batch) { return (batch + 127) / 128; }
 
 lt_status lt_dqueue_init(void* state, int L, int budget, int batch, lt_stream stream) {
+  LT_RANGE();
   if (!dq_args(state, L, batch) || budget < 0 || budget > L) return LT_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   lt_status st = device_info(&dev);
@@ -404,6 +424,7 @@ lt_status lt_dqueue_init(void* state, int L, int budget, int batch, lt_stream st
 
 lt_status lt_dqueue_push_gathered(void* state, int L, int batch, int layer, const float* ratio, int shards,
                                   int hq_shard, lt_stream stream) {
+  LT_RANGE();
   if (!dq_args(state, L, batch) || !aligned(ratio, 4) || shards < 1 || hq_shard < 1) return LT_ERR_INVALID_ARG;
   const cudaError_t e = launch_pdl(lt::dqueue_push_kernel, dim3(dq_blocks(batch)), dim3(128), 0,
                                    reinterpret_cast<cudaStream_t>(stream), state, L, batch, layer, ratio, hq_shard,
@@ -412,11 +433,13 @@ lt_status lt_dqueue_push_gathered(void* state, int L, int batch, int layer, cons
 }
 
 lt_status lt_dqueue_push(void* state, int L, int batch, int layer, const float* ratio, int hq, lt_stream stream) {
+  LT_RANGE();
   return lt_dqueue_push_gathered(state, L, batch, layer, ratio, 1, hq, stream);
 }
 
 lt_status lt_dqueue_result(const void* state, int L, int batch, int budget, uint8_t* lazy_mask, int32_t* order,
                            lt_stream stream) {
+  LT_RANGE();
   if (!dq_args(state, L, batch) || !lazy_mask || budget < 0 || budget > L || (order && !aligned(order, 4)))
     return LT_ERR_INVALID_ARG;
   lt::dqueue_result_kernel<<<dq_blocks(batch), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
@@ -425,6 +448,7 @@ lt_status lt_dqueue_result(const void* state, int L, int batch, int budget, uint
 }
 
 lt_status lt_dqueue_error(const void* state, int* error_bits) {
+  LT_RANGE();
   if (!aligned(state, 16) || !error_bits) return LT_ERR_INVALID_ARG;
   int32_t w = 0;
   if (cudaMemcpy(&w, static_cast<const int32_t*>(state) + 3, sizeof w, cudaMemcpyDeviceToHost) != cudaSuccess)
@@ -436,6 +460,7 @@ lt_status lt_dqueue_error(const void* state, int* error_bits) {
 lt_status lt_compact_kv_pending(const lt_shape* shape, const void* const* K_layers, const void* const* V_layers,
                                 const void* state, int L, int budget, int S, int W, void* K_pool, void* V_pool,
                                 int32_t* pool_len, lt_stream stream) {
+  LT_RANGE();
   lt_status st = check_shape(shape);
   if (st != LT_OK) return st;
   if (!aligned(K_layers, 8) || !aligned(V_layers, 8) || !dq_args(state, L, shape->batch) || budget < 1 ||
@@ -473,6 +498,7 @@ lt_status lt_compact_kv_pending(const lt_shape* shape, const void* const* K_laye
 
 lt_status lt_stream_ring_init(const int32_t* stream_len, int32_t* next_slot, int batch, int S, int W,
                               lt_stream stream) {
+  LT_RANGE();
   if (!aligned(stream_len, 4) || !aligned(next_slot, 4) || batch < 1 || S < 0 || W < 1) return LT_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   lt_status st = device_info(&dev);
@@ -484,6 +510,7 @@ lt_status lt_stream_ring_init(const int32_t* stream_len, int32_t* next_slot, int
 
 lt_status lt_stream_append(void* K_stream, void* V_stream, int32_t* stream_len, int32_t* next_slot, const void* k_new,
                            const void* v_new, int batch, int hkv, int head_dim, int S, int W, lt_stream stream) {
+  LT_RANGE();
   if (!aligned(K_stream, 16) || !aligned(V_stream, 16) || !aligned(stream_len, 4) || !aligned(next_slot, 4) ||
       !aligned(k_new, 16) || !aligned(v_new, 16) || batch < 1 || hkv < 1 || S < 0 || W < 1)
     return LT_ERR_INVALID_ARG;
@@ -539,6 +566,7 @@ lt_status launch_decode(lt::DecodeParams& p, int head_dim, int max_len, float so
 lt_status lt_stream_decode(const void* q, const void* K_stream, const void* V_stream, const int32_t* stream_len,
                            int batch, int hq, int hkv, int head_dim, int slots, void* O, float* LSE,
                            float softmax_scale, lt_stream stream) {
+  LT_RANGE();
   if (!aligned(q, 16) || !aligned(K_stream, 16) || !aligned(V_stream, 16) || !aligned(stream_len, 4) ||
       !aligned(O, 16) || !aligned(LSE, 4) || batch < 1 || batch > 65535 || hq < 1 || hkv < 1 || hq % hkv ||
       slots < 1 || !std::isfinite(softmax_scale))
@@ -565,6 +593,7 @@ lt_status lt_stream_decode(const void* q, const void* K_stream, const void* V_st
 lt_status lt_decode_attn(const void* q, const void* K, const void* V, const int32_t* seq_start, int seq_capacity,
                          const int32_t* len, int batch, int hq, int hkv, int head_dim, int max_len, void* O,
                          float* LSE, float softmax_scale, lt_stream stream) {
+  LT_RANGE();
   if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(len, 4) || !aligned(O, 16) ||
       !aligned(LSE, 4) || (seq_start && !aligned(seq_start, 4)) || batch < 1 || batch > 65535 || hq < 1 ||
       hkv < 1 || hq % hkv || max_len < 1 || (!seq_start && seq_capacity < max_len) ||
@@ -590,6 +619,7 @@ lt_status lt_decode_attn(const void* q, const void* K, const void* V, const int3
 }
 
 lt_status lt_selftest_wait_timeout(unsigned limit_us, lt_stream stream) {
+  LT_RANGE();
   if (limit_us == 0 || limit_us > 10000000u) return LT_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   lt_status st = device_info(&dev);
@@ -600,6 +630,7 @@ lt_status lt_selftest_wait_timeout(unsigned limit_us, lt_stream stream) {
 }
 
 lt_status lt_device_status(int clear) {
+  LT_RANGE();
   unsigned v = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return LT_ERR_CUDA;
   if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof v) != cudaSuccess) return LT_ERR_CUDA;
