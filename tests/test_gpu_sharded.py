@@ -205,3 +205,17 @@ def test_sequence_slices_match_full_batch(world):
             assert torch.equal(st.pool_len[:, i], full.pool_len[:, b])
             l0, l1, g0, g1 = local_cu[i], local_cu[i + 1], cu_h[b], cu_h[b + 1]
             assert torch.equal(st.O[l0:l1], full.O[g0:g1]) and torch.equal(st.LSE[:, l0:l1], full.LSE[:, g0:g1])
+
+
+def test_prefill_step_with_budget_zero_demotes_nothing():
+    cfg = _cfg()
+    step = lt.PrefillStep(_layers(cfg), 0, cfg.S, cfg.W, cfg.n_obs)
+    assert step.kernel_launches() == 1 + 2 * cfg.layers      # no compaction launches
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    step.enqueue(s)
+    torch.cuda.synchronize()
+    mask, order = step.dq.result()
+    torch.cuda.synchronize()
+    assert step.dq.error() == 0 and order.shape == (1, 0) and not bool(mask.any())
+    assert step.K_pool.numel() == 0
