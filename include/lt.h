@@ -37,7 +37,10 @@
  *     16-byte aligned.  When total_tokens is 0 the token-indexed inputs and
  *     outputs (Q, K, V, O, LSE) are not accessed and may be null.
  *   - Calls that take a stream only enqueue work on it (they never synchronise
- *     the device); their outputs are ready when the stream reaches them.
+ *     the device); their outputs are ready when the stream reaches them.  They
+ *     launch on the calling thread's current CUDA device: the stream and every
+ *     device pointer must belong to that device (the library cannot check a
+ *     pointer's device; the Python binding checks its tensors').
  *   - Arguments are checked before anything is enqueued.  A failed check returns
  *     LT_ERR_INVALID_ARG (or LT_ERR_UNSUPPORTED for a head_dim other than 64 or
  *     128) and enqueues nothing.  A launch failure returns LT_ERR_CUDA.
