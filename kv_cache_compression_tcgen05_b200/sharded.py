@@ -107,7 +107,9 @@ class PrefillStep:
     group of several ranks.  The per-layer Q/K/V stay owned by the caller; the
     step owns O/LSE scratch, the per-layer ratios, the device queue and the
     streaming-KV pool [budget, batch, hkv, S+W, d] of the demoted layers (this
-    rank's heads)."""
+    rank's heads).  The step's buffers are created on the current stream: a
+    step enqueued on another stream must be ordered after them and after the
+    inputs (e.g. stream.wait_stream(torch.cuda.current_stream()))."""
 
     def __init__(self, layers, budget, S, W, n_obs, cu_seqlens=None, max_seqlen=None, group=None):
         if not layers:
