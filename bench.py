@@ -112,6 +112,20 @@ def compaction_bytes(cfg, n_layers):
     return 2.0 * 2.0 * rows * cfg.hkv * cfg.d * 2 * n_layers
 
 
+def kv_fraction_after_prefill(order, pool_len, seqlens, layers):
+    """KV cache rows kept after the prefill over the rows of keeping every layer
+    full: per sequence b, the (layers - demoted) full layers keep N_b rows each
+    and each demoted layer the pool_len rows of its streaming cache.
+    order: [batch, budget] demoted layers (-1 past the count), pool_len:
+    [budget, batch] rows in demotion slot k; both host tensors."""
+    kept = total = 0
+    for b, n in enumerate(seqlens):
+        demoted = [k for k in range(order.shape[1]) if int(order[b, k]) >= 0]
+        kept += (layers - len(demoted)) * n + sum(int(pool_len[k, b]) for k in demoted)
+        total += layers * n
+    return kept / total if total else 1.0
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle samples while the timed region runs."""
 
@@ -306,6 +320,7 @@ def run_ours(args, cfg, rank, world):
         host_order.append([x for x in (q.push(l, lt.lt_layer_score(r[l, b])) for l in range(cfg.layers)) if x >= 0])
         q.close()
     queue_agrees = all(order_dev[b].tolist() == host_order[b] for b in range(lc.batch))
+    kv_frac = kv_fraction_after_prefill(order_dev.cpu(), pf.pool_len.cpu(), lc.seqlens, cfg.layers)
     ranks_agree = True
     if world > 1 and args.shard == "heads":
         orders = [torch.empty_like(order_dev) for _ in range(world)]
@@ -429,6 +444,7 @@ def run_ours(args, cfg, rank, world):
         "compaction_batched_gbs": round(compaction_bytes(lc, n_dem) / t_comp_batch / 1e9, 1),
         "separate_ratio_unique_gbs": round(ratio_unique_bytes(lc) / t_ratio / 1e9, 1),
         "device_queue_matches_host_queue": queue_agrees,
+        "kv_cache_fraction_after_prefill": round(kv_frac, 4),
         "ranks_demote_same_layers": ranks_agree,
         **decode,
         "roofline": {"kernel": "attn_fwd64_kernel (head_dim 64, fused with the lazy ratio)", "bound": "tensor",

@@ -1,7 +1,8 @@
 """Host logic of bench.py that the reported numbers rest on, checked without a GPU:
 the algorithmic work counts (closed forms against brute-force enumeration of
-the key sets the method defines) and the parsing of the nvidia-smi clock
-samples that decide whether a run is kept."""
+the key sets the method defines), the KV-cache fraction a prefill leaves
+(against the closed form (C + budget * min(1, (S+W)/N)) / L), and the parsing
+of the nvidia-smi clock samples that decide whether a run is kept."""
 import bench
 import synth
 
@@ -68,3 +69,24 @@ def test_clock_summary_reads_median_and_throttle_reasons():
     assert s["reasons"] == ["sw_power_cap"]
     cs.lines = ["0, 1500, 1965, 900, 0x8, Active, Not Active, Active, Not Active"]
     assert cs.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+
+
+def test_kv_fraction_after_prefill():
+    import torch
+    # one sequence, budget layers demoted, each keeping min(N, S+W) rows:
+    # (C + budget * min(1, (S+W)/N)) / L with C = L - budget
+    L, budget, N, S, W = 16, 8, 4096, 4, 1020
+    order = torch.arange(budget, dtype=torch.int32).reshape(1, budget)
+    pool_len = torch.full((budget, 1), min(N, S + W), dtype=torch.int32)
+    want = ((L - budget) + budget * min(1.0, (S + W) / N)) / L
+    assert abs(bench.kv_fraction_after_prefill(order, pool_len, (N,), L) - want) < 1e-12
+    assert want == 0.625
+    # ragged batch: sequence 1 demoted one layer only (-1 past its count), sequence 2 is short
+    order = torch.tensor([[3, 1], [2, -1], [0, 1]], dtype=torch.int32)
+    pool_len = torch.tensor([[24, 24, 9], [24, -7, 9]], dtype=torch.int32)    # [budget, batch]
+    seqlens, L = (100, 50, 9), 4
+    kept = (2 * 100 + 24 + 24) + (3 * 50 + 24) + (2 * 9 + 9 + 9)
+    assert abs(bench.kv_fraction_after_prefill(order, pool_len, seqlens, L) - kept / (L * 159)) < 1e-12
+    # budget 0: nothing demoted
+    empty = torch.zeros((2, 0), dtype=torch.int32)
+    assert bench.kv_fraction_after_prefill(empty, torch.zeros((0, 2), dtype=torch.int32), (5, 7), 3) == 1.0
