@@ -349,7 +349,7 @@ def run_ours(args, cfg, rank, world):
     if args.kernels_only:
         return {"metric": METRIC, "ms_per_step": round(ms, 4), "fused_us_per_layer": round(t_fused * 1e6, 2),
                 "attn_us_per_layer": round(t_attn * 1e6, 2), "ratio_us_per_layer": round(t_ratio * 1e6, 2),
-                "gpu_launches": launches}
+                "kv_cache_fraction_after_prefill": round(kv_frac, 4), "gpu_launches": launches}
 
     # Compaction timed on its own: every demoted layer of one step (inputs > L2 apart).
     mask1 = torch.ones(lc.batch, dtype=torch.uint8, device="cuda")
