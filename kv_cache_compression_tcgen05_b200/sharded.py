@@ -114,6 +114,10 @@ class PrefillStep:
     def __init__(self, layers, budget, S, W, n_obs, cu_seqlens=None, max_seqlen=None, group=None):
         if not layers:
             raise ValueError("at least one layer is required")
+        if any(len(lay) != 3 for lay in layers):
+            raise ValueError("every layer must be a (Q, K, V) triple")
+        if cu_seqlens is not None and max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
         Q0, K0, _ = layers[0]
         T, hq, d = Q0.shape
         hkv = K0.shape[1]

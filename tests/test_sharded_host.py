@@ -156,3 +156,16 @@ def test_pack_sequences_keeps_rows_and_lengths():
     packed, local_cu = lt.pack_sequences(t, cu, [2, 0])
     assert local_cu == [0, 5, 8]
     assert torch.equal(packed, torch.cat([t[7:12], t[0:3]]))
+
+
+def test_prefill_step_rejects_bad_layer_lists_before_allocating():
+    Q = torch.zeros((8, 4, 64), dtype=torch.bfloat16)
+    K = torch.zeros((8, 2, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        lt.PrefillStep([], 1, 4, 8, 4)
+    with pytest.raises(ValueError):
+        lt.PrefillStep([(Q, K)], 1, 4, 8, 4)
+    with pytest.raises(ValueError):
+        lt.PrefillStep([(Q, K, K), (Q, K, K[:4])], 1, 4, 8, 4)
+    with pytest.raises(ValueError):
+        lt.PrefillStep([(Q, K, K)], 1, 4, 8, 4, cu_seqlens=torch.tensor([0, 3, 8], dtype=torch.int32))
