@@ -4,7 +4,9 @@ ratios (with the oracle), all-gather them with the library's gather_ratios and
 run the library's host queue on the gathered scores; both ranks must demote the
 same layers as one process holding all heads, with bit-identical layer scores.
 Sequences: every sequence dealt to one rank, the slowest rank's work within the
-greedy bound, and packing of a rank's sequences."""
+greedy bound, and packing of a rank's sequences.  Failure: a rank that leaves
+before a layer's exchange makes the other rank's exchange fail with an error
+within the process group's timeout instead of hanging."""
 import os
 import socket
 
@@ -169,3 +171,38 @@ def test_prefill_step_rejects_bad_layer_lists_before_allocating():
         lt.PrefillStep([(Q, K, K), (Q, K, K[:4])], 1, 4, 8, 4)
     with pytest.raises(ValueError):
         lt.PrefillStep([(Q, K, K)], 1, 4, 8, 4, cu_seqlens=torch.tensor([0, 3, 8], dtype=torch.int32))
+
+
+def _rank_dies_main(rank, world, port, out):
+    import datetime
+    import time
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        os._exit(0)                       # leaves between steps, before the layer's exchange
+    gathered = torch.zeros((world, 1, 2))
+    t0 = time.monotonic()
+    try:
+        lt.gather_ratios(torch.ones((1, 2)), gathered)
+        out[rank] = ("no error", time.monotonic() - t0)
+    except RuntimeError as e:             # the exchange reports the missing rank
+        out[rank] = (type(e).__name__, time.monotonic() - t0)
+
+
+def test_exchange_fails_instead_of_hanging_when_a_rank_leaves():
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_dies_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=60)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:
+        p.kill()
+    assert not alive, "a rank hung on the exchange"
+    kind, seconds = out[0]
+    assert kind == "RuntimeError" and seconds < 30
