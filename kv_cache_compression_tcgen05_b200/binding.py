@@ -215,7 +215,7 @@ def lt_prefill_attn_ratio(Q, K, V, S, W, n_obs, cu_seqlens=None, max_seqlen=None
                                            out.data_ptr(), lse.data_ptr(),
                                            0.0 if softmax_scale is None else float(softmax_scale), int(S), int(W),
                                            int(n_obs), ratio.data_ptr(), _stream_handle(stream)),
-           "lt_prefill_attn_ratio")
+           "lt_prefill_attn_ratio_acc" if accumulate else "lt_prefill_attn_ratio")
     return out, lse, ratio
 
 
