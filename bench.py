@@ -1,17 +1,22 @@
 """Benchmark of the LightTransfer-Test prefill hot path.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config gqa1p2b] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config long128k] [--impl ours|reference]
 
 One step is one pass of the whole path over one prefill of the workload: for
-every layer the causal GQA attention with its LSE fused with the lazy ratio
-(lt_prefill_attn_ratio), the push of the layer's ratios into the device-resident
-layer queue (lt_dqueue_push) and the compaction of the layer the queue demotes,
-if any (lt_compact_kv_pending).  The whole step is one CUDA graph (no host round
-trip).  The per-layer Q/K/V of all layers are resident in HBM before timing
-(together far larger than the 126 MB L2, so no L2 flush is needed).  The plain
+every layer the causal GQA attention with its LSE fused with the lazy ratio and
+the push of the layer's ratios into the device-resident layer queue
+(lt_prefill_attn_ratio_push: the attention's last CTA pushes), then the
+compaction of the layer the queue demotes.  On the long-context workload
+(long128k, the default: the largest that one GPU holds, and the one whose
+prefill runs the queue online under the peak-memory cap) the step keeps the
+full KV of at most C + 1 layers: lt_kv_pool_commit reduces the demoted layer
+to its streaming rows and stores the current layer in the freed slot.  The
+whole step is one CUDA graph (no host round trip).  The per-layer Q/K/V of all
+layers are resident in HBM before timing (far larger than the 126 MB L2, so no
+L2 flush is needed between steps); in the capped mode they stand for the
+projections' outputs, each read only while its layer runs.  The plain
 attention (lt_prefill_attn), the separate ratio pass from the LSE
-(lt_lazy_ratio), the host queue and compaction (lt_compact_kv) are timed beside
-it.
+(lt_lazy_ratio) and compaction (lt_compact_kv) are timed beside it.
 
 Rank 0 prints one JSON line.  With --gpus N > 1 (torchrun) every rank runs an
 independent replica of the workload by default (--shard replicas): weak
@@ -46,7 +51,10 @@ import synth  # noqa: E402
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = "prefill attn+lazy-ratio TFLOP/s & % BF16 tensor peak; compaction GB/s; ratio ovh %"
 ATTN_SOURCES = ["kv_cache_compression_tcgen05_b200/csrc/attn_fwd64.cuh", "kv_cache_compression_tcgen05_b200/csrc/attn_fwd.cuh",
-                "kv_cache_compression_tcgen05_b200/csrc/lt_device.cuh"]
+                "kv_cache_compression_tcgen05_b200/csrc/lt_device.cuh", "kv_cache_compression_tcgen05_b200/csrc/dqueue.cuh"]
+# A per-launch time averaged over at least this long is taken under the
+# sustained (power-capped) tensor peak; shorter ones under the burst peak.
+SUSTAINED_REGION_S = 1.0
 
 
 def load_peaks():
@@ -66,10 +74,11 @@ def source_digest(paths):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(config_name):
-    """DRAM bytes per attention launch from the committed ncu summary, or None if
-    the kernel source changed since the counters were taken."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd64_{config_name}.traffic.txt")
+def recorded_traffic(config_name, d):
+    """DRAM bytes per attention launch from the committed ncu summary of the
+    head_dim-d kernel on this workload, or None if there is none or the kernel
+    source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd{d}_{config_name}.traffic.txt")
     if not os.path.exists(path):
         return None
     with open(path) as f:
@@ -110,6 +119,19 @@ def compaction_bytes(cfg, n_layers):
     """Bytes read + written by compacting n_layers demoted layers (K and V)."""
     rows = sum(min(n, cfg.S + cfg.W) for n in cfg.seqlens)
     return 2.0 * 2.0 * rows * cfg.hkv * cfg.d * 2 * n_layers
+
+
+def choose_peak(peaks, region_s):
+    """(peak TFLOP/s, source) for a kernel whose per-launch time was averaged
+    over region_s seconds of back-to-back work: the measured sustained bf16
+    peak (a seconds-long loop under the power cap) when that region lasts
+    seconds, else the burst peak."""
+    if region_s >= SUSTAINED_REGION_S:
+        return float(peaks["bf16_tflops_sustained"]), (
+            f"bf16_tflops_sustained: per-launch time averaged over {region_s:.1f} s of back-to-back launches "
+            f"(>= {SUSTAINED_REGION_S:.0f} s)")
+    return float(peaks["bf16_tflops"]), (
+        f"bf16_tflops (burst): per-launch time averaged over {region_s:.3f} s (< {SUSTAINED_REGION_S:.0f} s)")
 
 
 def kv_fraction_after_prefill(order, pool_len, seqlens, layers):
@@ -217,9 +239,10 @@ def barrier(world):
 class Prefill:
     """The whole path over every layer of one prefill, inputs resident on the GPU.
     With a process group the heads are split over its ranks (this rank's slice
-    of every layer's Q/K/V); otherwise this GPU holds all heads."""
+    of every layer's Q/K/V); otherwise this GPU holds all heads.  kv_pool: the
+    step keeps the full KV of at most C + 1 layers (the capped prefill)."""
 
-    def __init__(self, cfg, lt, device="cuda", group=None, seqs=None):
+    def __init__(self, cfg, lt, device="cuda", group=None, seqs=None, kv_pool=False):
         self.cfg, self.lt = cfg, lt
         if group is not None:
             q0, q1, k0, k1 = lt.head_shard(cfg.hq, cfg.hkv, torch.distributed.get_rank(group),
@@ -241,9 +264,15 @@ class Prefill:
                                          seqlens=tuple(cfg.seqlens[b] for b in self.seqs))
         lc = self.local
         cu = torch.tensor(lc.cu_seqlens(), dtype=torch.int32, device=device) if lc.batch > 1 else None
+        # Device memory the step itself takes (its buffers and anything it
+        # allocates while running), from here to the end of the first step.
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats()
+        self.mem_base = torch.cuda.memory_allocated()
         self.step = lt.PrefillStep(layers, cfg.budget, cfg.S, cfg.W, cfg.n_obs, cu_seqlens=cu,
-                                   max_seqlen=lc.max_seqlen, group=group)
+                                   max_seqlen=lc.max_seqlen, group=group, kv_pool=kv_pool)
         st = self.step
+        self.kv_pool = kv_pool
         self.layers, self.O, self.LSE, self.ratio = st.layers, st.O, st.LSE, st.ratio
         self.K_pool, self.V_pool, self.pool_len = st.K_pool, st.V_pool, st.pool_len
         self.Kp, self.Vp, self.dq, self.kw = st.Kp, st.Vp, st.dq, st.kw
@@ -253,24 +282,84 @@ class Prefill:
         pair of external timing events around every attention launch."""
         self.step.enqueue(stream, events=events)
 
+    def kv_report(self, step_alloc_bytes):
+        """The KV cache the step keeps (the method's memory outcome) and the
+        device memory the step took, measured by the allocator."""
+        st, cfg = self.step, self.local
+        full, stream, held = st.kv_bytes()
+        owned = sum(t.numel() * t.element_size() for t in (st.O, st.LSE, st.ratio, st.K_pool, st.V_pool,
+                                                            st.pool_len, st.dq.state))
+        if st.kv_pool:
+            owned += 2 * st.K_full.numel() * st.K_full.element_size()
+            peak = held + full            # the C slots, the working layer's own K/V, the streaming caches
+        else:
+            owned += 2 * st.Kp.numel() * 8
+            peak = cfg.layers * full + cfg.budget * stream   # every layer stays full in the caller's tensors
+        return {
+            "mode": ("capped: C = L - budget full-KV slots plus the working layer's K/V" if st.kv_pool else
+                     "every layer's full K/V resident (caller's tensors) plus the streaming caches"),
+            "full_layer_bytes": full, "stream_layer_bytes": stream,
+            "peak_kv_bytes": peak, "all_full_kv_bytes": cfg.layers * full,
+            "peak_kv_fraction_of_all_full": round(peak / (cfg.layers * full), 4),
+            "bound_bytes": (cfg.layers - cfg.budget + 1) * full + cfg.budget * stream,
+            "step_alloc_bytes_measured": int(step_alloc_bytes), "step_buffer_bytes": int(owned),
+        }
+
+
+def workload_config(cfg, kv_pool, world, shard):
+    """The `config` of the JSON line (both arms): the workload and how a step
+    runs it."""
+    import kv_cache_compression_tcgen05_b200 as lt
+    if shard == "heads":
+        q0, q1, k0, k1 = lt.head_shard(cfg.hq, cfg.hkv, 0, world)
+        par = (f"heads split over {world} rank(s): rank 0's q heads {q0}..{q1 - 1}, KV heads {k0}..{k1 - 1}; "
+               f"ratios all-gathered per layer (NCCL)")
+    elif shard == "sequences":
+        par = (f"sequences split over {world} rank(s) by causal work: rank 0's sequences "
+               f"{lt.sequence_shard(cfg.seqlens, 0, world)}; no exchange")
+    else:
+        par = f"replicas x{world}" if world > 1 else "single GPU"
+    return {
+        "workload": f"{cfg.name}: {cfg.layers} layers, batch {cfg.batch}, seq {cfg.max_seqlen}, "
+                    f"{cfg.hq} q heads / {cfg.hkv} KV heads, head_dim {cfg.d}, S={cfg.S}, W={cfg.W}, "
+                    f"n_obs={cfg.n_obs}, budget {cfg.budget}"
+                    + (", online queue under the peak-memory cap (C+1 full-KV layers)" if kv_pool else ""),
+        "layers": cfg.layers, "batch": cfg.batch, "seq_len": cfg.max_seqlen, "hq": cfg.hq, "hkv": cfg.hkv,
+        "head_dim": cfg.d, "S": cfg.S, "W": cfg.W, "n_obs": cfg.n_obs, "budget": cfg.budget,
+        "kv_pool": kv_pool,
+        "l2": "inputs of one step (all layers' Q/K/V) exceed L2; no flush between steps",
+        "step": "one CUDA graph: queue init, all layers' ratio accumulators zeroed once, then per layer fused "
+                "attention+ratio+queue push, then " + ("the slot commit (compaction of the demoted layer, "
+                                                       "store of the current one)" if kv_pool else
+                                                       "device-driven compaction")
+                + " (programmatic dependent launch)",
+        "parallelism": par,
+    }
+
 
 def run_ours(args, cfg, rank, world):
     import kv_cache_compression_tcgen05_b200 as lt
     lt.library()
     peaks, peak_src = load_peaks()
     sharded = args.shard != "replicas"
+    kv_pool = cfg.online if args.kv_pool == "auto" else args.kv_pool == "on"
     pf = Prefill(cfg, lt, group=torch.distributed.group.WORLD if args.shard == "heads" else None,
-                 seqs=lt.sequence_shard(cfg.seqlens, rank, world) if args.shard == "sequences" else None)
+                 seqs=lt.sequence_shard(cfg.seqlens, rank, world) if args.shard == "sequences" else None,
+                 kv_pool=kv_pool)
     lc = pf.local   # this rank's shape: all heads and sequences, or its slice when sharded
     stream = torch.cuda.Stream()
     stream.wait_stream(torch.cuda.current_stream())   # the inputs were made on the default stream
+    t0 = time.perf_counter()
     with torch.cuda.stream(stream):
         pf.enqueue_step(stream)           # eager warm-up: per-device set-up happens outside capture
     torch.cuda.synchronize()
+    t_eager = time.perf_counter() - t0
+    step_alloc = torch.cuda.max_memory_allocated() - pf.mem_base
     if args.decode_only:
         # One prefill step for the demotions, then the decode leg alone (a
         # short command for profiling the decode kernel).
         return {"metric": "decode after prefill", "config": cfg.name, **measure_decode(lc, lt, pf, peaks)}
+    long_step = t_eager > 0.5             # seconds-long steps: fewer repetitions beside the timed region
     g_step = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step, stream=stream):
         pf.enqueue_step(stream)
@@ -285,7 +374,7 @@ def run_ours(args, cfg, rank, world):
     g_events = torch.cuda.CUDAGraph()
     fused_ev = []
     with torch.cuda.graph(g_events, stream=stream):
-        for _ in range(2):
+        for _ in range(1 if long_step else 2):
             pf.enqueue_step(stream, events=fused_ev)
     for _ in range(args.warmup):
         g_step.replay()
@@ -304,9 +393,13 @@ def run_ours(args, cfg, rank, world):
     barrier(world)
     launches = args.steps * pf.step.kernel_launches()
     ms = max_over_ranks(start.elapsed_time(stop), world) / args.steps
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
+        ev0.record(stream)
         g_events.replay()
+        ev1.record(stream)
     torch.cuda.synchronize()
+    events_region_s = ev0.elapsed_time(ev1) * 1e-3
     del g_step, g_timed, g_events   # before any process-group teardown (they may hold NCCL calls)
     t_fused = statistics.mean(a.elapsed_time(b) for a, b in fused_ev) * 1e-3
     # The demotions of the timed steps equal the host queue's on the same ratios
@@ -327,29 +420,35 @@ def run_ours(args, cfg, rank, world):
         torch.distributed.all_gather(orders, order_dev.contiguous())
         ranks_agree = all(torch.equal(o, orders[0]) for o in orders)
 
-    # Beside the step: the plain attention and the separate ratio pass per layer.
+    # Beside the step: the plain attention and the separate ratio pass per
+    # layer (all layers twice for short steps, the first four once for long ones).
     kw = pf.kw
+    side_layers = list(range(min(cfg.layers, 4))) if long_step else list(range(cfg.layers))
     attn_ev, ratio_ev = [], []
-    for rep in range(2):
-        for l in range(cfg.layers):
+    ratio_out = torch.empty_like(pf.ratio[0])
+    for rep in range(2 if not long_step else 1):
+        for l in side_layers:
             Q, K, V = pf.layers[l]
             e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
             e0.record()
             lt.lt_prefill_attn(Q, K, V, out=pf.O, lse=pf.LSE, **kw)
             e1.record()
-            lt.lt_lazy_ratio(Q, K, pf.LSE, cfg.S, cfg.W, cfg.n_obs, out=pf.ratio[l], **kw)
+            lt.lt_lazy_ratio(Q, K, pf.LSE, cfg.S, cfg.W, cfg.n_obs, out=ratio_out, **kw)
             e2.record()
-            if rep > 0:
+            if rep > 0 or long_step and l > 0:
                 attn_ev.append((e0, e1))
                 ratio_ev.append((e1, e2))
     torch.cuda.synchronize()
     t_attn = statistics.mean(a.elapsed_time(b) for a, b in attn_ev) * 1e-3
     t_ratio = statistics.mean(a.elapsed_time(b) for a, b in ratio_ev) * 1e-3
+    kv = pf.kv_report(step_alloc)
 
     if args.kernels_only:
-        return {"metric": METRIC, "ms_per_step": round(ms, 4), "fused_us_per_layer": round(t_fused * 1e6, 2),
+        return {"metric": METRIC, "config": {"workload": cfg.name, "kv_pool": kv_pool},
+                "ms_per_step": round(ms, 4), "fused_us_per_layer": round(t_fused * 1e6, 2),
                 "attn_us_per_layer": round(t_attn * 1e6, 2), "ratio_us_per_layer": round(t_ratio * 1e6, 2),
-                "kv_cache_fraction_after_prefill": round(kv_frac, 4), "gpu_launches": launches}
+                "kv_cache_fraction_after_prefill": round(kv_frac, 4), "kv_cache": kv, "gpu_launches": launches,
+                "events_region_s": round(events_region_s, 3)}
 
     # Compaction timed on its own: every demoted layer of one step (inputs > L2 apart).
     mask1 = torch.ones(lc.batch, dtype=torch.uint8, device="cuda")
@@ -371,12 +470,14 @@ def run_ours(args, cfg, rank, world):
     _, order_now = pf.dq.result()
     demoted_layers = order_now[0].to(torch.int32).contiguous()
     n_dem = int((demoted_layers >= 0).sum())
+    Kp = pf.Kp if pf.Kp is not None else lt.layer_pointer_table([lay[1] for lay in pf.layers])
+    Vp = pf.Vp if pf.Vp is not None else lt.layer_pointer_table([lay[2] for lay in pf.layers])
     cb_times = []
     for rep in range(6):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        lt.lt_compact_kv_layers(pf.Kp, pf.Vp, demoted_layers, lc.S, lc.W, pf.K_pool, pf.V_pool, pf.pool_len,
+        lt.lt_compact_kv_layers(Kp, Vp, demoted_layers, lc.S, lc.W, pf.K_pool, pf.V_pool, pf.pool_len,
                                 lc.total_tokens, lc.hkv, lc.d, **kw)
         e1.record()
         torch.cuda.synchronize()
@@ -385,6 +486,10 @@ def run_ours(args, cfg, rank, world):
     del flush
     t_comp = statistics.mean(c_times)
     t_comp_batch = statistics.median(cb_times)
+    # The step's own buffers (pools, queue) hold its result again for the legs below.
+    with torch.cuda.stream(stream):
+        pf.enqueue_step(stream)
+    torch.cuda.synchronize()
 
     # Per-kernel figures are this rank's; the job is world whole prefills
     # (replicas) or the one prefill split over the ranks.
@@ -392,15 +497,17 @@ def run_ours(args, cfg, rank, world):
     job_flops = cfg.layers * (attention_flops(cfg) + ratio_flops(cfg)) * (1 if sharded else world)
     value = job_flops / (ms * 1e-3) / 1e12
     achieved = fl_attn / t_fused / 1e12
-    peak_sus = float(peaks["bf16_tflops_sustained"])
+    peak, peak_why = choose_peak(peaks, events_region_s)
     peak_burst = float(peaks["bf16_tflops"])
-    traffic = recorded_traffic(cfg.name) if lc == cfg else None   # the record is of the all-heads launch
+    traffic = recorded_traffic(cfg.name, cfg.d) if lc == cfg else None   # the record is of the all-heads launch
     comp_gbs = compaction_bytes(lc, 1) / t_comp / 1e9
 
     decode = measure_decode(lc, lt, pf, peaks)
-    e2e = measure_e2e(args, lc, lt, pf, world, job_flops)
+    e2e = measure_e2e(args, lc, lt, pf, world, job_flops, long_step)
     cpu = cpu_baseline(cfg) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     clocks = clk.summary()
+    kernel = (f"attn_fwd64_kernel<fused> (head_dim 64, fused with the lazy ratio and the queue push)" if cfg.d == 64
+              else f"attn_fwd_kernel<128, fused> (head_dim 128, fused with the lazy ratio and the queue push)")
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -413,23 +520,9 @@ def run_ours(args, cfg, rank, world):
         "scaling": "strong" if sharded else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16 Q/K/V with per-layer sink bias; pages' datasets/weights absent)",
-        "config": {
-            "workload": f"{cfg.name}: {cfg.layers} layers, batch {cfg.batch}, seq {cfg.max_seqlen}, "
-                        f"{cfg.hq} q heads / {cfg.hkv} KV heads, head_dim {cfg.d}, S={cfg.S}, W={cfg.W}, "
-                        f"n_obs={cfg.n_obs}, budget {cfg.budget}",
-            "layers": cfg.layers, "batch": cfg.batch, "seq_len": cfg.max_seqlen, "hq": cfg.hq, "hkv": cfg.hkv,
-            "head_dim": cfg.d, "S": cfg.S, "W": cfg.W, "n_obs": cfg.n_obs, "budget": cfg.budget,
-            "l2": "inputs of one step (all layers' Q/K/V) exceed L2; no flush between steps",
-            "step": "one CUDA graph: queue init, all layers' ratio accumulators zeroed once, then per layer fused "
-                    "attention+ratio, device queue push, device-driven compaction (programmatic dependent launch)",
-            "parallelism": (f"heads split over {world} rank(s): this rank's q heads {pf.heads[0]}..{pf.heads[1] - 1}, "
-                            f"KV heads {pf.heads[2]}..{pf.heads[3] - 1}; ratios all-gathered per layer (NCCL)"
-                            if args.shard == "heads" else
-                            f"sequences split over {world} rank(s) by causal work: rank 0's sequences {pf.seqs}; "
-                            f"no exchange" if args.shard == "sequences" else
-                            f"replicas x{world}" if world > 1 else "single GPU"),
-        },
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V with per-layer sink and recency biases; pages' datasets/weights "
+                "absent)",
+        "config": workload_config(cfg, kv_pool, world, args.shard),
         "attn_tflops": round(achieved, 2),
         "attn_pct_of_burst_peak": round(100 * achieved / peak_burst, 2),
         "fused_attn_ratio_us_per_layer": round(t_fused * 1e6, 2),
@@ -445,12 +538,14 @@ def run_ours(args, cfg, rank, world):
         "separate_ratio_unique_gbs": round(ratio_unique_bytes(lc) / t_ratio / 1e9, 1),
         "device_queue_matches_host_queue": queue_agrees,
         "kv_cache_fraction_after_prefill": round(kv_frac, 4),
+        "kv_cache": kv,
         "ranks_demote_same_layers": ranks_agree,
         **decode,
-        "roofline": {"kernel": "attn_fwd64_kernel (head_dim 64, fused with the lazy ratio)", "bound": "tensor",
-                     "achieved": round(achieved, 2), "peak": peak_sus, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak_sus, 4), "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step)"},
+        "roofline": {"kernel": kernel, "bound": "tensor",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "frac_of_burst": round(achieved / peak_burst, 4),
+                     "traffic": traffic, "peak_source": f"{peak_src} {peak_why}",
+                     "algorithmic_flop_per_launch": fl_attn},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
@@ -478,9 +573,19 @@ def measure_decode(cfg, lt, pf, peaks):
     lens = torch.tensor([cu_h[b + 1] - cu_h[b] for b in range(B)], dtype=torch.int32, device="cuda")
     stream = torch.cuda.Stream()
 
+    # Kept layers read their full cache: the layer's own tensors, or its
+    # full-KV slot in the capped mode.
+    slots = pf.dq.slots() if pf.kv_pool else None
+    full_cache = {}
+    for l in range(cfg.layers):
+        if pf.kv_pool and l in slot_of:
+            continue
+        K, V, st = pf.step.kept_layer_cache(l, slots)
+        full_cache[l] = (K, V, st if pf.kv_pool else starts)
+
     def full(l, s):
-        _, K, V = pf.layers[l]
-        lt.lt_decode_attn(q, K, V, lens, seq_start=starts, max_len=cfg.max_seqlen, out=O, lse=LSE, stream=s)
+        K, V, st = full_cache[l] if l in full_cache else (pf.layers[l][1], pf.layers[l][2], starts)
+        lt.lt_decode_attn(q, K, V, lens, seq_start=st, max_len=cfg.max_seqlen, out=O, lse=LSE, stream=s)
 
     def streaming(l, s):
         k = slot_of[l]
@@ -519,7 +624,7 @@ def measure_decode(cfg, lt, pf, peaks):
 
     t_hybrid = timed(hybrid_step)
     t_full = timed(full_step)
-    t_full_layer = timed(lambda s: full(0, s), reps=20)
+    t_full_layer = timed(lambda s: full(min(full_cache) if full_cache else 0, s), reps=20)
     t_stream_layer = timed(lambda s: streaming(demoted[0], s), reps=20) if demoted else None
     del flush
     n_rows = sum(cu_h[b + 1] - cu_h[b] for b in range(B))
@@ -543,43 +648,50 @@ def measure_decode(cfg, lt, pf, peaks):
     return out
 
 
-def measure_e2e(args, cfg, lt, pf, world, job_flops):
+def measure_e2e(args, cfg, lt, pf, world, job_flops, long_step):
     """Same metric through the public calls with host buffers: every step copies
-    each layer's Q/K/V from pinned host memory to the device and reads back each
-    layer's O and LSE, the ratios and the streaming KV pool, all inside the
-    device-timed region.  Uploads run one layer ahead on a side stream and
-    read-backs on another, so copies overlap the kernels; the queue lives on the
-    device, so no step waits for the host.  The full K/V of every layer stay on
-    the device (the KV cache the queue manages); Q is double buffered.  `cfg` is
-    this rank's shape (its slice when the heads or sequences are split);
+    each layer's Q/K/V from pinned host memory to the device and reads back the
+    step's result -- the last layer's O and LSE, every layer's ratios and the
+    demoted layers' streaming KV with its lengths -- all inside the
+    device-timed region.  Uploads run one layer ahead on a side stream (two
+    device buffers for Q, each reused every other layer) and the read-back on
+    another, so copies overlap the kernels; the queue lives on the device, so
+    no step waits for the host.  In the capped mode K/V take the same two
+    device buffers (the step keeps its own C full-KV slots); otherwise every
+    layer's K/V stays on the device (the KV cache the queue manages).  `cfg`
+    is this rank's shape (its slice when the heads or sequences are split);
     job_flops the work of the whole job per step."""
-    host = [tuple(t.cpu().pin_memory() for t in lay) for lay in pf.layers]
+    host = []
+    for lay in pf.layers:
+        host.append(tuple(torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t) for t in lay))
     T, H, d = cfg.total_tokens, cfg.hq, cfg.d
     dev_q = [torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-    dev_kv = [tuple(torch.empty_like(t) for t in lay[1:]) for lay in pf.layers]
+    if pf.kv_pool:
+        bufs = [tuple(torch.empty_like(t) for t in pf.layers[0][1:]) for _ in range(2)]
+        dev_kv = [bufs[l % 2] for l in range(cfg.layers)]
+    else:
+        dev_kv = [tuple(torch.empty_like(t) for t in lay[1:]) for lay in pf.layers]
     step = lt.PrefillStep([(dev_q[l % 2],) + dev_kv[l] for l in range(cfg.layers)], cfg.budget, cfg.S, cfg.W,
-                          cfg.n_obs, group=pf.step.group, **pf.kw)
-    o_host = torch.empty((cfg.layers, T, H, d), dtype=torch.bfloat16, pin_memory=True)
-    lse_host = torch.empty((cfg.layers, H, T), dtype=torch.float32, pin_memory=True)
+                          cfg.n_obs, group=pf.step.group, kv_pool=pf.kv_pool, **pf.kw)
+    o_host = torch.empty((T, H, d), dtype=torch.bfloat16, pin_memory=True)
+    lse_host = torch.empty((H, T), dtype=torch.float32, pin_memory=True)
     ratio_host = torch.empty(step.ratio.shape, dtype=torch.float32, pin_memory=True)
     ks_host = torch.empty(step.K_pool.shape, dtype=torch.bfloat16, pin_memory=True)
     vs_host = torch.empty_like(ks_host)
-    O = [torch.empty((T, H, d), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-    LSE = [torch.empty((H, T), dtype=torch.float32, device="cuda") for _ in range(2)]
+    len_host = torch.empty(step.pool_len.shape, dtype=torch.int32, pin_memory=True)
     copy_in, copy_out = torch.cuda.Stream(), torch.cuda.Stream()
     main = torch.cuda.current_stream()
     h2d = sum(t.numel() * t.element_size() for lay in host for t in lay)
-    d2h = o_host.numel() * 2 + lse_host.numel() * 4 + ratio_host.numel() * 4 + 2 * ks_host.numel() * 2
+    d2h = sum(t.numel() * t.element_size() for t in (o_host, lse_host, ratio_host, ks_host, vs_host, len_host))
 
     def one_step():
         ready = [torch.cuda.Event() for _ in range(cfg.layers)]
-        done = [torch.cuda.Event() for _ in range(cfg.layers)]
         computed = [torch.cuda.Event() for _ in range(cfg.layers)]
 
         def upload(l):
             with torch.cuda.stream(copy_in):
                 if l >= 2:
-                    copy_in.wait_event(done[l - 2])   # Q buffer and O/LSE of layer l-2 consumed
+                    copy_in.wait_event(computed[l - 2])   # layer l-2 no longer reads these buffers
                 dev_q[l % 2].copy_(host[l][0], non_blocking=True)
                 dev_kv[l][0].copy_(host[l][1], non_blocking=True)
                 dev_kv[l][1].copy_(host[l][2], non_blocking=True)
@@ -591,65 +703,85 @@ def measure_e2e(args, cfg, lt, pf, world, job_flops):
             if l + 1 < cfg.layers:
                 upload(l + 1)
             main.wait_event(ready[l])
-            step.layer(l, main, O=O[l % 2], LSE=LSE[l % 2])
+            step.layer(l, main)
             computed[l].record(main)
-            with torch.cuda.stream(copy_out):
-                copy_out.wait_event(computed[l])
-                o_host[l].copy_(O[l % 2], non_blocking=True)
-                lse_host[l].copy_(LSE[l % 2], non_blocking=True)
-                done[l].record(copy_out)
         with torch.cuda.stream(copy_out):
             copy_out.wait_stream(main)
+            o_host.copy_(step.O, non_blocking=True)
+            lse_host.copy_(step.LSE, non_blocking=True)
             ratio_host.copy_(step.ratio, non_blocking=True)
             ks_host.copy_(step.K_pool, non_blocking=True)
             vs_host.copy_(step.V_pool, non_blocking=True)
+            len_host.copy_(step.pool_len, non_blocking=True)
         main.wait_stream(copy_out)
         main.wait_stream(copy_in)
 
-    for _ in range(2):
+    for _ in range(1 if long_step else 2):
         one_step()
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    steps = max(1, min(args.steps, 5))
+    steps = max(1, min(args.steps, 2 if long_step else 5))
     e0.record()
     for _ in range(steps):
         one_step()
     e1.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    ok = bool(torch.equal(step.ratio, pf.step.ratio))     # same result as the device-resident step
     return {"value": round(job_flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 3)}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 3),
+            "steps": steps, "ratios_match_device_inputs_step": ok}
 
 
 # ------------------------------------------------------------- CPU (oracle)
 
+_ORACLE_INPUTS = {}
+
+
 def oracle_sample(cfg, seconds, seed=0):
-    """Time the fp64 oracle on a bounded random sample of the workload's rows:
-    attention rows (uniform over tokens and heads) of layer 0 plus the lazy
-    ratio of a proportional share of the observed rows.  Returns
-    (TFLOP/s, cores, description)."""
+    """Time the fp64 oracle, as it stands, on a bounded random sample of one
+    layer's work in the metric's unit (algorithmic attention + lazy-ratio
+    FLOPs per second): random (token, head) attention rows of layer 0 and
+    random (observed row, head) lazy-ratio rows of layer 0, the latter in
+    the proportion of the layer's ratio FLOPs to its attention FLOPs (at least
+    one).  The oracle's ratio row takes its LSE from a full attention row
+    (route A without a given LSE), so it costs about as much as one.
+    Returns (TFLOP/s, cores, description)."""
     import oracle
-    Q, K, V = synth.layer_inputs(cfg, 0, "cpu")
-    q, k, v = synth.bf16_bits(Q), synth.bf16_bits(K), synth.bf16_bits(V)
+    if cfg.name not in _ORACLE_INPUTS:   # drawn once per process: a long workload's layer takes seconds on the host
+        _ORACLE_INPUTS.clear()
+        _ORACLE_INPUTS[cfg.name] = tuple(synth.bf16_bits(t) for t in synth.layer_inputs(cfg, 0, "cpu"))
+    q, k, v = _ORACLE_INPUTS[cfg.name]
     cu = np.array(cfg.cu_seqlens(), np.int32)
     cores = os.cpu_count() or 1
     rng = np.random.default_rng(seed)
     starts = np.array(cfg.cu_seqlens()[:-1])
+    obs = [(cu[b] + i, i) for b, n in enumerate(cfg.seqlens) for i in range(n - min(cfg.n_obs, n), n)]
+    share = ratio_flops(cfg) / attention_flops(cfg)
 
     def run(n):
         toks = rng.integers(0, cfg.total_tokens, n).astype(np.int32)
         heads = rng.integers(0, cfg.hq, n).astype(np.int32)
         pos = toks - starts[np.searchsorted(starts, toks, side="right") - 1]
+        n_r = max(1, int(round(n * share)))
+        pick = rng.integers(0, len(obs), n_r)
+        rt = np.array([obs[i][0] for i in pick], np.int32)
+        rp = np.array([obs[i][1] for i in pick], np.int64)
+        rh = rng.integers(0, cfg.hq, n_r).astype(np.int32)
         t0 = time.perf_counter()
         oracle.attn(cu, q, k, v, tokens=toks, heads=heads, nthreads=cores)
+        oracle.lazy_ratio_rows(cu, q, k, cfg.S, cfg.W, rt, rh, nthreads=cores)
         t = time.perf_counter() - t0
-        return 4.0 * cfg.d * float(np.sum(pos + 1)), t
+        fl = 4.0 * cfg.d * float(np.sum(pos + 1))
+        fl += 2.0 * cfg.d * float(np.sum(np.minimum(cfg.S + cfg.W, rp + 1)))
+        return fl, t, n, n_r
 
-    fl, t = run(64)
+    fl, t, _, _ = run(64)
     n = int(min(200000, max(64, 64 * seconds / max(t, 1e-3))))
-    fl, t = run(n)
-    return fl / t / 1e12, cores, f"{n} random (token, head) attention rows of layer 0 ({fl / 1e9:.1f} GFLOP, {t:.1f} s)"
+    fl, t, n, n_r = run(n)
+    return fl / t / 1e12, cores, (f"{n} random (token, head) attention rows and {n_r} random observed (row, head) "
+                                  f"lazy-ratio rows of layer 0 ({fl / 1e9:.1f} GFLOP, {t:.1f} s)")
 
 
 def cpu_baseline(cfg, seconds=10.0):
@@ -662,11 +794,12 @@ def run_reference(args, cfg, rank, world):
         return None
     vals = []
     desc = ""
+    oracle_sample(cfg, 0.1, seed=0)        # draws the inputs once, outside the timed steps
     for _ in range(args.warmup):
-        oracle_sample(cfg, 2.0, seed=1)
+        oracle_sample(cfg, 1.0, seed=1)
     t0 = time.perf_counter()
     for s in range(args.steps):
-        v, cores, desc = oracle_sample(cfg, 5.0, seed=100 + s)
+        v, cores, desc = oracle_sample(cfg, 4.0, seed=100 + s)
         vals.append(v)
     ms = (time.perf_counter() - t0) * 1e3 / max(1, args.steps)
     value = statistics.mean(vals)
@@ -674,9 +807,10 @@ def run_reference(args, cfg, rank, world):
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{cfg.name} (fp64 CPU oracle on a bounded random row sample per step)"},
+        "config": workload_config(cfg, cfg.online if args.kv_pool == "auto" else args.kv_pool == "on", world,
+                                  args.shard),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+                         "sample": f"each step: {desc}; the fp64 oracle on the host cores"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -686,7 +820,12 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", default="gqa1p2b")
+    ap.add_argument("--config", default="long128k",
+                    help="workload (synth.CONFIGS); long128k is the largest that one GPU holds")
+    ap.add_argument("--kv-pool", default="auto", choices=["auto", "on", "off"],
+                    help="keep the full KV of at most C+1 layers (auto: on for the online, memory-capped workload)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="a smaller case: only the workload's first N layers (budget scaled to N); for profiling")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-only", action="store_true",
@@ -701,6 +840,10 @@ def main():
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     cfg = synth.CONFIGS[args.config]
+    if args.layers:
+        n = max(1, min(args.layers, cfg.layers))
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}-first{n}layers", layers=n,
+                                  budget=int(round(cfg.budget * n / cfg.layers)))
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         line = run_reference(args, cfg, rank, args.gpus)

@@ -134,6 +134,24 @@ lt_status lt_prefill_attn_ratio_acc(const lt_shape* shape, const void* Q, const 
                                     lt_stream stream);
 
 /*
+ * lt_prefill_attn_ratio_acc followed, inside the same kernel, by the
+ * device-queue push of this layer (lt_dqueue_push(state, L, batch, layer,
+ * ratio, hq)): the last CTA of the attention to finish -- after every CTA has
+ * added its share of the ratios -- pushes each sequence's score, so a layer of
+ * the prefill costs one launch fewer.  ratio must be zero on entry (as for
+ * lt_prefill_attn_ratio_acc); state, L and the push's rule, slots and errors
+ * are those of lt_dqueue_push.  If the attention gives up a bounded wait the
+ * push is skipped, no layer is recorded as demoted by it and the queue's
+ * error bit 4 is set (lt_dqueue_error).  With no tokens the push still
+ * happens (every ratio 0).  The state also holds the launch's completion
+ * counter: two launches that use the same state must not overlap.
+ * Sources: as lt_prefill_attn_ratio and lt_dqueue_push.
+ */
+lt_status lt_prefill_attn_ratio_push(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
+                                     float* LSE, float softmax_scale, int S, int W, int n_obs, float* ratio,
+                                     void* state, int L, int layer, lt_stream stream);
+
+/*
  * Lazy ratio from the LSE.
  *   For every sequence b (length N), query head h and each of the last
  *   n' = min(n_obs, N) rows i of b:
@@ -142,7 +160,8 @@ lt_status lt_prefill_attn_ratio_acc(const lt_shape* shape, const void* Q, const 
  *   ratio[b, h] = mean of r_i over those rows (0 when N == 0).
  * Q, K as for lt_prefill_attn; LSE: device fp32 [hq, T] as written by it.
  * ratio: device fp32 [batch, hq] (written).  S >= 0, W >= 0, S + W >= 1,
- * 1 <= n_obs <= 4096.
+ * 1 <= n_obs <= 4096; hq and batch at most 65535 (one cluster of CTAs per
+ * (sequence, query head)).  Deterministic: the same inputs give the same bits.
  * Sources: the press-release page's definition (attention weights to the
  * initial and recent keys) and the write-up's first solution (LSE as the
  * denominator; O(S+W) work per query).
@@ -159,7 +178,8 @@ float lt_layer_score(const float* ratio_of_heads, int hq);
  * sequence the layers are ranked by (score descending, layer ascending) and
  * the first `budget` are lazy.  lazy_mask: host uint8 [batch, L] (written, 0/1);
  * order: host int32 [batch, budget] (nullable; written in rank order).
- * 0 <= budget <= L.  Scores that are NaN are rejected.  Host-only, synchronous.
+ * 0 <= budget <= L.  A non-finite score (NaN or +-inf) is rejected with
+ * LT_ERR_INVALID_ARG, as lt_queue_push rejects it.  Host-only, synchronous.
  */
 lt_status lt_select_layers(const float* ratios, int L, int batch, int hq, int budget, uint8_t* lazy_mask,
                            int32_t* order);
@@ -221,7 +241,14 @@ lt_status lt_compact_kv_layers(const lt_shape* shape, const void* const* K_layer
  * as lt_layer_score does, so host and device queues demote the same layers.
  *
  * state: caller-allocated device memory of lt_dqueue_state_bytes(L, batch)
- * bytes, 16-byte aligned; lt_dqueue_init (re)initialises it on `stream`.
+ * bytes (4 * (8 + 3 batch + 5 batch L)), 16-byte aligned; lt_dqueue_init
+ * (re)initialises it on `stream`.
+ *
+ * The queue also assigns full-KV slots for a memory-capped prefill
+ * (lt_kv_pool_commit): each queued layer owns one of C = L - budget slots.
+ * A pushed layer takes a never-used slot (slot n-1 for the n-th queued
+ * layer) while no layer has been demoted, afterwards the slot of the layer
+ * its push demotes, or none when it is demoted by its own push.
  * lt_dqueue_push: ratio is device fp32 [batch, hq] (e.g. the ratio output of
  * lt_prefill_attn_ratio for this layer).  A push that is invalid for a
  * sequence (layer out of range or pushed twice, non-finite score) leaves that
@@ -252,7 +279,12 @@ lt_status lt_dqueue_push_gathered(void* state, int L, int batch, int layer, cons
                                   int hq_shard, lt_stream stream);
 lt_status lt_dqueue_result(const void* state, int L, int batch, int budget, uint8_t* lazy_mask, int32_t* order,
                            lt_stream stream);
+/* Error bits of the queue (synchronous): 1 an invalid push, 2 a call whose
+ * L / batch differ from init's, 4 a fused push skipped (lt_prefill_attn_ratio_push). */
 lt_status lt_dqueue_error(const void* state, int* error_bits);
+/* slots: device int32 [batch, L] (written): the full-KV slot of each layer of
+ * each sequence, -1 for a layer that holds none (demoted, or not pushed). */
+lt_status lt_dqueue_slots(const void* state, int L, int batch, int32_t* slots, lt_stream stream);
 
 /*
  * Compaction driven by the device queue: for every sequence b whose latest
@@ -269,6 +301,37 @@ lt_status lt_dqueue_error(const void* state, int* error_bits);
 lt_status lt_compact_kv_pending(const lt_shape* shape, const void* const* K_layers, const void* const* V_layers,
                                 const void* state, int L, int budget, int S, int W, void* K_pool, void* V_pool,
                                 int32_t* pool_len, lt_stream stream);
+
+/*
+ * One layer of the prefill under the peak-memory cap: "the layer with the
+ * highest ratio is made lazy and its KV cache reduced, freeing memory for
+ * storing the KV cache of the current layer" (project page, Methodology,
+ * LightTransfer-Test, Figure 2 caption; the write-up's second solution:
+ * at most 50% full KV + 50% streaming KV at the prefill's peak).  Enqueue it
+ * right after the push of `layer` (lt_dqueue_push or
+ * lt_prefill_attn_ratio_push).  For every sequence b:
+ *   - if the push demoted a layer m (the k-th demotion of b), m's streaming
+ *     rows p = [0, min(S,N)) ++ [max(S, N-W), N) are written to streaming slot
+ *     k (as lt_compact_kv_pending; zero past the kept count, stream_len[k, b]
+ *     = |p|), read from K_cur/V_cur when m == layer, else from m's full-KV slot;
+ *   - if the current layer holds a full-KV slot s after the push (it was not
+ *     demoted), its rows are stored there: K_full[s, cu[b] + r] = K_cur[cu[b] + r]
+ *     for every r < N (same for V) -- when m != layer, s is the slot m just
+ *     released, and m's kept rows are read before they are overwritten.
+ * K_cur, V_cur: device bf16 [T, hkv, d], the current layer's K/V in a buffer of
+ * the caller's (read only; with the full-KV slots, at most C + 1 layers' full
+ * KV exist at once).  K_full, V_full: device bf16 [L - budget, T, hkv, d]
+ * (unused when budget == L).  K_stream, V_stream: device bf16
+ * [budget, batch, hkv, S+W, d]; stream_len: device int32 [budget, batch]
+ * (unused when budget == 0).  The layer -> slot map is read back with
+ * lt_dqueue_slots (e.g. for decode of the full layers: sequence b's rows of
+ * layer l start at row slot * T + cu[b] of K_full viewed as [(L-budget) T, hkv, d]).
+ * Errors: LT_ERR_INVALID_ARG for a bad shape, state size, layer or window, or
+ * misaligned buffers.  Asynchronous on `stream`; nothing is allocated.
+ */
+lt_status lt_kv_pool_commit(const lt_shape* shape, const void* K_cur, const void* V_cur, const void* state, int L,
+                            int budget, int layer, int S, int W, void* K_full, void* V_full, void* K_stream,
+                            void* V_stream, int32_t* stream_len, lt_stream stream);
 
 /*
  * Decode on a demoted layer's streaming KV cache (press-release page: the

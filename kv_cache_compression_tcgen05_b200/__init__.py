@@ -27,6 +27,7 @@ from .binding import (  # noqa: F401
     lt_lazy_ratio,
     lt_prefill_attn,
     lt_prefill_attn_ratio,
+    lt_prefill_attn_ratio_push,
     lt_queue_create,
     lt_queue_destroy,
     lt_queue_push,
@@ -45,7 +46,9 @@ from .binding import (  # noqa: F401
     lt_dqueue_push,
     lt_dqueue_push_gathered,
     lt_dqueue_result,
+    lt_dqueue_slots,
     lt_dqueue_state_bytes,
+    lt_kv_pool_commit,
     lt_stream_append,
     lt_stream_decode,
     lt_decode_attn,

@@ -48,6 +48,7 @@ _SIGS = {
     "lt_prefill_attn": (_i, [_shp, _vp, _vp, _vp, _vp, _vp, _f, _vp]),
     "lt_prefill_attn_ratio": (_i, [_shp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
     "lt_prefill_attn_ratio_acc": (_i, [_shp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
+    "lt_prefill_attn_ratio_push": (_i, [_shp, _vp, _vp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp, _i, _i, _vp]),
     "lt_lazy_ratio": (_i, [_shp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
     "lt_layer_score": (_f, [_vp, _i]),
     "lt_select_layers": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
@@ -64,6 +65,8 @@ _SIGS = {
     "lt_dqueue_error": (_i, [_vp, ctypes.POINTER(_i)]),
     "lt_compact_kv_pending": (_i, [_shp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "lt_compact_kv_layers": (_i, [_shp, _vp, _vp, _i, _vp, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "lt_kv_pool_commit": (_i, [_shp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "lt_dqueue_slots": (_i, [_vp, _i, _i, _vp, _vp]),
     "lt_stream_ring_init": (_i, [_vp, _vp, _i, _i, _i, _vp]),
     "lt_stream_append": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "lt_stream_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp]),
@@ -216,6 +219,38 @@ def lt_prefill_attn_ratio(Q, K, V, S, W, n_obs, cu_seqlens=None, max_seqlen=None
                                            0.0 if softmax_scale is None else float(softmax_scale), int(S), int(W),
                                            int(n_obs), ratio.data_ptr(), _stream_handle(stream)),
            "lt_prefill_attn_ratio_acc" if accumulate else "lt_prefill_attn_ratio")
+    return out, lse, ratio
+
+
+def lt_prefill_attn_ratio_push(Q, K, V, S, W, n_obs, queue, layer, ratio, cu_seqlens=None, max_seqlen=None,
+                               softmax_scale=None, out=None, lse=None, stream=None):
+    """Attention fused with the lazy ratio and the device-queue push of `layer`
+    (see include/lt.h): ratio [batch, hq] must be zero on entry; queue is a
+    DeviceQueue.  Returns (O, LSE, ratio)."""
+    _dev_tensor(Q, "Q", torch.bfloat16, 3)
+    _dev_tensor(K, "K", torch.bfloat16, 3)
+    _dev_tensor(V, "V", torch.bfloat16, 3)
+    T, hq, d = Q.shape
+    hkv = K.shape[1]
+    if K.shape != (T, hkv, d) or V.shape != K.shape:
+        raise ValueError("K and V must be [T, hkv, d] with Q's T and d")
+    shape = _shape(T, hq, hkv, d, cu_seqlens, max_seqlen)
+    if shape.batch != queue.batch:
+        raise ValueError("batch differs from the queue's")
+    if out is None:
+        out = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty((hq, T), dtype=torch.float32, device=Q.device)
+    _sized(out, "out", torch.bfloat16, (T, hq, d))
+    _sized(lse, "lse", torch.float32, (hq, T))
+    _sized(ratio, "ratio", torch.float32, (shape.batch, hq))
+    _dev_tensor(queue.state, "state", torch.uint8, 1)
+    _check(library().lt_prefill_attn_ratio_push(ctypes.byref(shape), Q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                                out.data_ptr(), lse.data_ptr(),
+                                                0.0 if softmax_scale is None else float(softmax_scale), int(S),
+                                                int(W), int(n_obs), ratio.data_ptr(), queue.state.data_ptr(),
+                                                queue.L, int(layer), _stream_handle(stream)),
+           "lt_prefill_attn_ratio_push")
     return out, lse, ratio
 
 
@@ -425,6 +460,9 @@ class DeviceQueue:
     def error(self) -> int:
         return lt_dqueue_error(self.state)
 
+    def slots(self, stream=None):
+        return lt_dqueue_slots(self.state, self.L, self.batch, stream=stream)
+
 
 def layer_pointer_table(tensors, device="cuda"):
     """Device int64 array of the tensors' data pointers (for lt_compact_kv_pending)."""
@@ -475,6 +513,45 @@ def lt_compact_kv_layers(K_layers, V_layers, layers, S, W, K_pool, V_pool, pool_
     _check(library().lt_compact_kv_layers(ctypes.byref(shape), K_layers.data_ptr(), V_layers.data_ptr(), L,
                                           layers.data_ptr(), n, int(S), int(W), K_pool.data_ptr(), V_pool.data_ptr(),
                                           pool_len.data_ptr(), _stream_handle(stream)), "lt_compact_kv_layers")
+
+
+def lt_kv_pool_commit(K_cur, V_cur, queue, layer, S, W, K_full, V_full, K_stream, V_stream, stream_len,
+                      cu_seqlens=None, max_seqlen=None, stream=None):
+    """One layer of the memory-capped prefill after its push (see include/lt.h):
+    the demoted layer's streaming rows into its streaming slot, the current
+    layer's K/V (K_cur, V_cur [T, hkv, d]) into its full-KV slot.
+    K_full / V_full [L - budget, T, hkv, d]; K_stream / V_stream
+    [budget, batch, hkv, S+W, d]; stream_len [budget, batch]."""
+    _dev_tensor(K_cur, "K_cur", torch.bfloat16, 3)
+    _dev_tensor(V_cur, "V_cur", torch.bfloat16, 3)
+    T, hkv, d = K_cur.shape
+    if V_cur.shape != K_cur.shape:
+        raise ValueError("V_cur must match K_cur")
+    shape = _shape(T, hkv, hkv, d, cu_seqlens, max_seqlen)
+    if shape.batch != queue.batch:
+        raise ValueError("batch differs from the queue's")
+    L, budget, B, slots = queue.L, queue.budget, queue.batch, int(S) + int(W)
+    _sized(K_full, "K_full", torch.bfloat16, (L - budget, T, hkv, d))
+    _sized(V_full, "V_full", torch.bfloat16, (L - budget, T, hkv, d))
+    _sized(K_stream, "K_stream", torch.bfloat16, (budget, B, hkv, slots, d))
+    _sized(V_stream, "V_stream", torch.bfloat16, (budget, B, hkv, slots, d))
+    _sized(stream_len, "stream_len", torch.int32, (budget, B))
+    _dev_tensor(queue.state, "state", torch.uint8, 1)
+    _check(library().lt_kv_pool_commit(ctypes.byref(shape), K_cur.data_ptr(), V_cur.data_ptr(),
+                                       queue.state.data_ptr(), L, budget, int(layer), int(S), int(W),
+                                       K_full.data_ptr(), V_full.data_ptr(), K_stream.data_ptr(), V_stream.data_ptr(),
+                                       stream_len.data_ptr(), _stream_handle(stream)), "lt_kv_pool_commit")
+
+
+def lt_dqueue_slots(state, L, batch, out=None, stream=None):
+    """Full-KV slot of every layer of every sequence: device int32 [batch, L] (-1: none)."""
+    _dev_tensor(state, "state", torch.uint8, 1)
+    if out is None:
+        out = torch.empty((batch, L), dtype=torch.int32, device=state.device)
+    _sized(out, "out", torch.int32, (batch, L))
+    _check(library().lt_dqueue_slots(state.data_ptr(), int(L), int(batch), out.data_ptr(), _stream_handle(stream)),
+           "lt_dqueue_slots")
+    return out
 
 
 def lt_stream_ring_init(stream_len, next_slot, S, W, stream=None):

@@ -49,6 +49,7 @@
 // two-term sum does not depend on the order.
 #pragma once
 
+#include "dqueue.cuh"
 #include "lt_device.cuh"
 
 namespace lt {
@@ -72,6 +73,11 @@ struct AttnParams {
   int S;
   int W;
   int n_obs;
+  // fused device-queue push (null: none): after every CTA has added its
+  // ratios, the last one pushes layer dq_layer's scores into the queue state
+  void* dq_state;
+  int dq_L;
+  int dq_layer;
 };
 
 template <int D>
@@ -426,10 +432,33 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
         }
         l_run *= alpha;
         if constexpr (kRatio) num *= alpha;
+        const float neg_m = -m_run;
+        // Fused ratio: the weights of the keys in K_i = [0, min(S, i+1)) U
+        // [max(S, i-W+1), i] within this key tile (columns c = key - 128 j).
+        // Keys after i carry weight 0 (causal mask), so a tile that starts
+        // inside the window counts whole (its row sum, below); only the tile
+        // holding the window's first key and the tile holding the sinks need
+        // a per-key mask.  That masked sum is taken before P is built, so the
+        // scores die as the exponential loop consumes them in every tile.
+        bool whole = false, part = false;
+        if constexpr (kRatio) {
+          const int win_c = qpos - p.W + 1 - j * 128;   // first window column
+          const int sink_c = p.S - j * 128;              // columns below it are sinks
+          whole = row_obs && win_c <= 0;
+          part = row_obs && !whole && (win_c < 128 || sink_c > 0);
+          if (__any_sync(0xffffffffu, part)) {
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+              const float w = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, neg_m));
+              acc += (c < sink_c || c >= win_c) ? w : 0.f;
+            }
+            if (part) num += acc;
+          }
+        }
         // exp2 in 32-column chunks; each chunk's bf16 P goes to TMEM (16
         // columns) as soon as it is packed.
         float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const float neg_m = -m_run;
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
           uint32_t pk[16];
@@ -449,25 +478,7 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
             ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
         l_run += tile_sum;
         if constexpr (kRatio) {
-          // Weights of the keys in K_i = [0, min(S, i+1)) U [max(S, i-W+1), i]
-          // within this key tile (columns c = key - 128 j).  Keys after i carry
-          // weight 0 (causal mask), so a tile that starts inside the window
-          // counts whole; only the tile holding the window's first key and the
-          // tile holding the sinks need a per-key mask.
-          const int win_c = qpos - p.W + 1 - j * 128;   // first window column
-          const int sink_c = p.S - j * 128;              // columns below it are sinks
-          const bool whole = row_obs && win_c <= 0;
-          const bool part = row_obs && !whole && (win_c < 128 || sink_c > 0);
           if (whole) num += tile_sum;
-          if (__any_sync(0xffffffffu, part)) {
-            float acc = 0.f;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-              const float w = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, neg_m));
-              acc += (c < sink_c || c >= win_c) ? w : 0.f;
-            }
-            if (part) num += acc;
-          }
         }
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // PV(j-1) is complete (S(j) was issued after it by the same thread):
@@ -543,6 +554,12 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, Lay::kTmemCols);
+  }
+  if constexpr (kRatio) {
+    // Fused queue push: the last CTA to finish pushes every sequence's score.
+    if (p.dq_state)
+      dq_last_cta_push(p.dq_state, p.dq_L, p.batch, p.dq_layer, p.ratio, p.hq, *abort_flag != 0,
+                       reinterpret_cast<int*>(smem + Lay::kMiscOff + 56));
   }
 }
 

@@ -340,27 +340,22 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[x]);
         const float neg_m = -m_run;
+        // Fused ratio: the weights of the keys in K_i = [0, min(S, i+1)) U
+        // [max(S, i-W+1), i] within this key tile (columns c = key - 128 j).
+        // Keys after i carry weight 0 (causal mask), so a tile that starts
+        // inside the window counts whole (its row sum, below); only the tile
+        // holding the window's first key and the tile holding the sinks need
+        // a per-key mask, which the exponential loop applies to the weights it
+        // computes anyway (a second instance of the loop, taken warp-uniformly
+        // by those tiles only: no exponential is evaluated twice).
+        int win_c = 0, sink_c = 0;
+        bool whole = false, part = false;
         if constexpr (kRatio) {
-          // Weights of the keys in K_i = [0, min(S, i+1)) U [max(S, i-W+1), i]
-          // within this key tile (columns c = key - 128 j).  Keys after i carry
-          // weight 0 (causal mask), so a tile that starts inside the window
-          // counts whole (added below, from the tile's row sum); only the tile
-          // holding the window's first key and the tile holding the sinks need
-          // a per-key mask.  Done before P so the scores die as P is built.
-          const int win_c = qpos - p.W + 1 - j * 128;   // first window column
-          const int sink_c = p.S - j * 128;              // columns below it are sinks
-          const bool whole = row_obs && win_c <= 0;
-          const bool part = row_obs && !whole && (win_c < 128 || sink_c > 0);
-          if (__any_sync(0xffffffffu, part)) {
-            float acc = 0.f;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-              const float w = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, neg_m));
-              acc += (c < sink_c || c >= win_c) ? w : 0.f;
-            }
-            if (part) num += acc;
-          }
-          }
+          win_c = qpos - p.W + 1 - j * 128;   // first window column
+          sink_c = p.S - j * 128;              // columns below it are sinks
+          whole = row_obs && win_c <= 0;
+          part = row_obs && !whole && (win_c < 128 || sink_c > 0);
+        }
         // P_x(j) in four 32-column chunks of bf16 pairs; the first two are
         // held in registers and written with the third.  Before the first
         // write, P_x(j-1) V_{j-1} must be done with the P columns (and with O,
@@ -370,40 +365,58 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
         // that PV time to finish.
         float2 sum4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float2 sl2x2 = make_float2(sl2, sl2), neg_mx2 = make_float2(neg_m, neg_m);
-        uint32_t pk0[16], pk1[16];
+        auto exp_tile = [&](auto masked_tag) -> float {
+          constexpr bool kMasked = decltype(masked_tag)::value;
+          float2 msum = make_float2(0.f, 0.f);
+          uint32_t pk0[16], pk1[16];
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-          uint32_t pk[16];
+          for (int cb = 0; cb < 4; ++cb) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int c0 = cb * 32 + 2 * c;
-            const float2 xx = fma_f32x2(make_float2(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1])), sl2x2,
-                                        neg_mx2);
-            // kPolyPairs of every 16 pairs go to the FMA pipe, the rest to MUFU.
-            const bool poly = (c & 15) >= 16 - kPolyPairs;
-            const float p0 = poly ? exp2_fma(xx.x) : fast_exp2(xx.x);
-            const float p1 = poly ? exp2_fma(xx.y) : fast_exp2(xx.y);
-            sum4[c & 3] = add_f32x2(sum4[c & 3], make_float2(p0, p1));
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-          if (cb == 2 && j > 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], cnt_pv & 1, ctl));
-            ++cnt_pv;
-            tc_fence_after();
-          }
-          if (cb == 0) {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) pk0[c] = pk[c];
-          } else if (cb == 1) {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) pk1[c] = pk[c];
-          } else {
-            if (cb == 2) {
-              tmem_st16(p_col, pk0);
-              tmem_st16(p_col + 16, pk1);
+            for (int c = 0; c < 16; ++c) {
+              const int c0 = cb * 32 + 2 * c;
+              const float2 xx = fma_f32x2(make_float2(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1])),
+                                          sl2x2, neg_mx2);
+              // kPolyPairs of every 16 pairs go to the FMA pipe, the rest to MUFU.
+              const bool poly = (c & 15) >= 16 - kPolyPairs;
+              const float p0 = poly ? exp2_fma(xx.x) : fast_exp2(xx.x);
+              const float p1 = poly ? exp2_fma(xx.y) : fast_exp2(xx.y);
+              sum4[c & 3] = add_f32x2(sum4[c & 3], make_float2(p0, p1));
+              if constexpr (kMasked) {
+                msum.x += (c0 < sink_c || c0 >= win_c) ? p0 : 0.f;
+                msum.y += (c0 + 1 < sink_c || c0 + 1 >= win_c) ? p1 : 0.f;
+              }
+              pk[c] = pack_bf16x2(p0, p1);
             }
-            tmem_st16(p_col + cb * 16, pk);
+            if (cb == 2 && j > 0) {
+              ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], cnt_pv & 1, ctl));
+              ++cnt_pv;
+              tc_fence_after();
+            }
+            if (cb == 0) {
+#pragma unroll
+              for (int c = 0; c < 16; ++c) pk0[c] = pk[c];
+            } else if (cb == 1) {
+#pragma unroll
+              for (int c = 0; c < 16; ++c) pk1[c] = pk[c];
+            } else {
+              if (cb == 2) {
+                tmem_st16(p_col, pk0);
+                tmem_st16(p_col + 16, pk1);
+              }
+              tmem_st16(p_col + cb * 16, pk);
+            }
           }
+          return msum.x + msum.y;
+        };
+        float part_sum = 0.f;
+        if constexpr (kRatio) {
+          if (__any_sync(0xffffffffu, part))
+            part_sum = exp_tile(std::true_type{});
+          else
+            exp_tile(std::false_type{});
+        } else {
+          exp_tile(std::false_type{});
         }
         if (!ok) break;
         const float2 s01 = add_f32x2(sum4[0], sum4[1]), s23 = add_f32x2(sum4[2], sum4[3]);
@@ -411,7 +424,8 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
         const float tile_sum = s0123.x + s0123.y;
         l_run += tile_sum;
         if constexpr (kRatio) {
-          if (row_obs && qpos - p.W + 1 - j * 128 <= 0) num += tile_sum;
+          if (whole) num += tile_sum;
+          if (part) num += part_sum;
         }
         if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
@@ -492,6 +506,12 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, Lay::kTmemCols);
+  }
+  if constexpr (kRatio) {
+    // Fused queue push: the last CTA to finish pushes every sequence's score.
+    if (p.dq_state)
+      dq_last_cta_push(p.dq_state, p.dq_L, p.batch, p.dq_layer, p.ratio, p.hq, *abort_flag != 0,
+                       reinterpret_cast<int*>(smem + Lay::kMiscOff + 56));
   }
 }
 

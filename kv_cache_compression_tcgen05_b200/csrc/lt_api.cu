@@ -74,9 +74,9 @@ lt_status device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(lt::attn_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              lt::AttnLayout<128>::kAlloc) != cudaSuccess ||
         cudaFuncSetAttribute(lt::lazy_ratio_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             lt::RatioLayout<64>::bytes(lt::kRatioMaxGroup * 256)) != cudaSuccess ||
+                             lt::RatioLayout<64>::kBytes) != cudaSuccess ||
         cudaFuncSetAttribute(lt::lazy_ratio_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             lt::RatioLayout<128>::bytes(lt::kRatioMaxGroup * 256)) != cudaSuccess)
+                             lt::RatioLayout<128>::kBytes) != cudaSuccess)
       return LT_ERR_CUDA;
     // Clusters of 16 CTAs are beyond the portable size: use them for the decode
     // split only where the device reports that one fits.
@@ -176,9 +176,13 @@ extern "C" {
 
 // Shared by lt_prefill_attn and lt_prefill_attn_ratio: checks, descriptors,
 // launch.  `ratio` null selects the plain attention kernel.
+static bool dq_args(const void* state, int L, int batch);
+static int dq_blocks(int batch);
+
 static lt_status launch_attention(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
                                   float* LSE, float softmax_scale, int S, int W, int n_obs, float* ratio,
-                                  lt_stream stream, bool zero_ratio = true) {
+                                  lt_stream stream, bool zero_ratio = true, void* dq_state = nullptr,
+                                  int dq_L = 0, int dq_layer = 0) {
   lt_status st = check_shape(shape);
   if (st != LT_OK) return st;
   if (!std::isfinite(softmax_scale)) return LT_ERR_INVALID_ARG;
@@ -189,6 +193,8 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (T > 0 && (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) || !aligned(LSE, 4)))
     return LT_ERR_INVALID_ARG;
+  if (dq_state && (!ratio || !dq_args(dq_state, dq_L, shape->batch) || dq_layer < 0 || dq_layer >= dq_L))
+    return LT_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   if (ratio && zero_ratio) {
     // The kernel adds each tile's share of the mean; sequences without tokens keep 0.
@@ -197,7 +203,14 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
     if (launch_pdl(lt::zero_f32_kernel, dim3((n + 255) / 256), dim3(256), 0, s, ratio, n) != cudaSuccess)
       return LT_ERR_CUDA;
   }
-  if (T == 0 || max_len == 0) return LT_OK;  // nothing to read or write
+  if (T == 0 || max_len == 0) {
+    // Nothing to read or write; the queue still takes the layer (all ratios 0).
+    if (!dq_state) return LT_OK;
+    const cudaError_t e = launch_pdl(lt::dqueue_push_kernel, dim3(dq_blocks(shape->batch)), dim3(128), 0, s,
+                                     dq_state, dq_L, shape->batch, dq_layer, static_cast<const float*>(ratio),
+                                     shape->hq, 1);
+    return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
+  }
   const int group = shape->hq / shape->hkv;
   const long long n_qtiles = (max_len + 127) / 128;
   const bool pair_heads = (group % 2) == 0;
@@ -230,6 +243,9 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
   p.S = S;
   p.W = W;
   p.n_obs = n_obs;
+  p.dq_state = dq_state;
+  p.dq_L = dq_L;
+  p.dq_layer = dq_layer;
   const int grid = int(num_items < dev->sm_count ? num_items : dev->sm_count);
   cudaError_t e;
   if (d == 64) {
@@ -270,6 +286,14 @@ lt_status lt_prefill_attn_ratio_acc(const lt_shape* shape, const void* Q, const 
   return launch_attention(shape, Q, K, V, O, LSE, softmax_scale, S, W, n_obs, ratio, stream, false);
 }
 
+lt_status lt_prefill_attn_ratio_push(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O,
+                                     float* LSE, float softmax_scale, int S, int W, int n_obs, float* ratio,
+                                     void* state, int L, int layer, lt_stream stream) {
+  LT_RANGE();
+  if (!ratio || !state) return LT_ERR_INVALID_ARG;
+  return launch_attention(shape, Q, K, V, O, LSE, softmax_scale, S, W, n_obs, ratio, stream, false, state, L, layer);
+}
+
 lt_status lt_lazy_ratio(const lt_shape* shape, const void* Q, const void* K, const float* LSE, float softmax_scale,
                         int S, int W, int n_obs, float* ratio, lt_stream stream) {
   LT_RANGE();
@@ -281,7 +305,7 @@ lt_status lt_lazy_ratio(const lt_shape* shape, const void* Q, const void* K, con
   if (S < 0 || W < 0 || (long long)S + W < 1 || n_obs < 1 || n_obs > 4096) return LT_ERR_INVALID_ARG;
   if (!std::isfinite(softmax_scale)) return LT_ERR_INVALID_ARG;
   const int group = shape->hq / shape->hkv;
-  if (group > lt::kRatioMaxGroup) return LT_ERR_UNSUPPORTED;
+  if (shape->hq > 65535 || shape->batch > 65535) return LT_ERR_INVALID_ARG;
 
   DeviceInfo* dev = nullptr;
   if ((st = device_info(&dev)) != LT_OK) return st;
@@ -301,15 +325,14 @@ lt_status lt_lazy_ratio(const lt_shape* shape, const void* Q, const void* K, con
   p.scale_log2 = resolve_scale(softmax_scale, shape->head_dim) * kLog2e;
   p.ratio = ratio;
 
-  // Cluster size: enough CTAs that each stages about 64 or more keys of the band.
+  // Cluster size: about kRatioKeysPerCta keys of the longest sequence's band per CTA.
   const long long max_len = shape->cu_seqlens ? shape->max_seqlen : shape->total_tokens;
   const long long band = std::min<long long>(S, max_len) + std::min<long long>(max_len, (long long)n_obs + W - 1);
-  int cluster = int(std::min<long long>(lt::kRatioMaxCluster, std::max<long long>(1, (band + 63) / 64)));
-  p.n_units = group * ((n_obs + 15) / 16);
-  const int warps = std::max(4, std::min(lt::kRatioMaxWarps, p.n_units));
+  const int cluster = int(std::min<long long>(
+      lt::kRatioMaxCluster, std::max<long long>(1, (band + lt::kRatioKeysPerCta - 1) / lt::kRatioKeysPerCta)));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cluster, shape->hkv, shape->batch);
-  cfg.blockDim = dim3(32 * warps, 1, 1);
+  cfg.gridDim = dim3(cluster, shape->hq, shape->batch);
+  cfg.blockDim = dim3(32 * lt::kRatioWarps, 1, 1);
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -320,10 +343,10 @@ lt_status lt_lazy_ratio(const lt_shape* shape, const void* Q, const void* K, con
   cfg.numAttrs = 1;
   cudaError_t e;
   if (shape->head_dim == 64) {
-    cfg.dynamicSmemBytes = lt::RatioLayout<64>::bytes(p.n_units);
+    cfg.dynamicSmemBytes = lt::RatioLayout<64>::kBytes;
     e = cudaLaunchKernelEx(&cfg, lt::lazy_ratio_kernel<64>, p);
   } else {
-    cfg.dynamicSmemBytes = lt::RatioLayout<128>::bytes(p.n_units);
+    cfg.dynamicSmemBytes = lt::RatioLayout<128>::kBytes;
     e = cudaLaunchKernelEx(&cfg, lt::lazy_ratio_kernel<128>, p);
   }
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
@@ -409,7 +432,7 @@ static bool dq_args(const void* state, int L, int batch) {
   return aligned(state, 16) && L >= 1 && L <= 4096 && batch >= 1 && batch <= (1 << 20);
 }
 
-static int dq_blocks(int batch) { return (batch + 127) / 128; }
+static int dq_blocks(int batch) { return (batch + 3) / 4; }   // 128 threads: a warp per sequence
 
 lt_status lt_dqueue_init(void* state, int L, int budget, int batch, lt_stream stream) {
   LT_RANGE();
@@ -493,6 +516,62 @@ lt_status lt_compact_kv_pending(const lt_shape* shape, const void* const* K_laye
   if (launch_pdl(lt::compact_pending_kernel, dim3(int(blocks)), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream),
                  p) != cudaSuccess)
     return LT_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_kv_pool_commit(const lt_shape* shape, const void* K_cur, const void* V_cur, const void* state, int L,
+                            int budget, int layer, int S, int W, void* K_full, void* V_full, void* K_stream,
+                            void* V_stream, int32_t* stream_len, lt_stream stream) {
+  LT_RANGE();
+  lt_status st = check_shape(shape);
+  if (st != LT_OK) return st;
+  if (!dq_args(state, L, shape->batch) || budget < 0 || budget > L || layer < 0 || layer >= L) return LT_ERR_INVALID_ARG;
+  if (S < 0 || W < 0 || (long long)S + W < 1 || (long long)S + W > (1 << 24)) return LT_ERR_INVALID_ARG;
+  if (shape->total_tokens > 0 && (!aligned(K_cur, 16) || !aligned(V_cur, 16))) return LT_ERR_INVALID_ARG;
+  if (budget < L && shape->total_tokens > 0 && (!aligned(K_full, 16) || !aligned(V_full, 16)))
+    return LT_ERR_INVALID_ARG;
+  if (budget > 0 && (!aligned(K_stream, 16) || !aligned(V_stream, 16) || !aligned(stream_len, 4)))
+    return LT_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if ((st = device_info(&dev)) != LT_OK) return st;
+  lt::PoolCommitParams p;
+  p.batch = shape->batch;
+  p.total_tokens = shape->total_tokens;
+  p.hkv = shape->hkv;
+  p.D = shape->head_dim;
+  p.S = S;
+  p.W = W;
+  p.L = L;
+  p.budget = budget;
+  p.layer = layer;
+  p.cu_seqlens = shape->cu_seqlens;
+  p.K_cur = static_cast<const uint4*>(K_cur);
+  p.V_cur = static_cast<const uint4*>(V_cur);
+  p.K_full = static_cast<uint4*>(K_full);
+  p.V_full = static_cast<uint4*>(V_full);
+  p.state = state;
+  p.K_stream = static_cast<uint4*>(K_stream);
+  p.V_stream = static_cast<uint4*>(V_stream);
+  p.stream_len = stream_len;
+  // Enough CTAs to stream a whole layer's K/V at HBM bandwidth.
+  const long long work = std::max<long long>((long long)shape->total_tokens, (long long)shape->batch * (S + W)) *
+                         shape->hkv * (shape->head_dim / 8);
+  long long blocks = (work + 255) / 256;
+  const long long cap = (long long)dev->sm_count * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  if (launch_pdl(lt::kv_pool_commit_kernel, dim3(int(blocks)), dim3(256), 0, reinterpret_cast<cudaStream_t>(stream),
+                 p) != cudaSuccess)
+    return LT_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_dqueue_slots(const void* state, int L, int batch, int32_t* slots, lt_stream stream) {
+  LT_RANGE();
+  if (!dq_args(state, L, batch) || !aligned(slots, 4)) return LT_ERR_INVALID_ARG;
+  const long long n = (long long)batch * L;
+  const int blocks = int(std::min<long long>((n + 127) / 128, 4096));
+  lt::dqueue_slots_kernel<<<blocks, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(state, L, batch, slots);
   return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
 }
 

@@ -291,7 +291,8 @@ __device__ __forceinline__ float exp2_fma(float x) {
                        0.9999289512634277f);
   // The low bits of t's representation hold round(x) (two's complement within
   // the mantissa); shifted by 23 they become round(x) in the exponent field.
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  // Unsigned arithmetic: the shift drops t's own exponent bits (mod 2^32).
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 // max(a, b, c) in one instruction (three-input max of sm_100).

@@ -114,7 +114,7 @@ lt_status lt_select_layers(const float* ratios, int L, int batch, int hq, int bu
   for (int b = 0; b < batch; ++b) {
     for (int l = 0; l < L; ++l) {
       score[l] = lt_layer_score(ratios + (size_t(l) * batch + b) * hq, hq);
-      if (std::isnan(score[l])) return LT_ERR_INVALID_ARG;
+      if (!std::isfinite(score[l])) return LT_ERR_INVALID_ARG;   // as lt_queue_push
     }
   }
   for (int b = 0; b < batch; ++b) {

@@ -104,33 +104,79 @@ class PrefillStep:
 
     layers: one (Q [T, hq, d], K [T, hkv, d], V [T, hkv, d]) bf16 device tuple
     per layer -- all heads, or this rank's head slice when `group` is a process
-    group of several ranks.  The per-layer Q/K/V stay owned by the caller; the
-    step owns O/LSE scratch, the per-layer ratios, the device queue and the
-    streaming-KV pool [budget, batch, hkv, S+W, d] of the demoted layers (this
-    rank's heads).  The step's buffers are created on the current stream: a
-    step enqueued on another stream must be ordered after them and after the
+    group of several ranks.  The per-layer Q/K/V stay owned by the caller.
+
+    Two ways to keep the KV cache (LightTransfer project page, Methodology,
+    LightTransfer-Test, Figure 2 caption; the write-up's second solution):
+
+    * kv_pool=False: every layer's full K/V stays in the caller's tensors; a
+      demoted layer's streaming rows are gathered into the streaming pool
+      (lt_compact_kv_pending) and the caller may release its full K/V.
+    * kv_pool=True (the prefill under the peak-memory cap): the step owns a
+      pool of C = L - budget full-KV slots [C, T, hkv, d].  A layer's K/V is
+      read from the caller's tensors only while the layer runs; after its
+      queue push, lt_kv_pool_commit reduces the demoted layer to its
+      streaming rows and stores the current layer in the slot that freed (or
+      a never-used one), unless the current layer was demoted itself.  At
+      most C + 1 layers' full K/V then exist at any time: the C slots and the
+      current layer's own buffer, so the caller can produce every layer's K/V
+      into one working buffer.  An entry of `layers` may then be None, with
+      the layer's tensors handed to layer(..., qkv=) and `dims` = (T, hq,
+      hkv, d) giving the shapes.
+
+    The step owns O/LSE scratch, the per-layer ratios, the device queue and
+    the streaming-KV pool [budget, batch, hkv, S+W, d] of the demoted layers
+    (this rank's heads).  Without a process group the queue push rides on the
+    attention kernel (lt_prefill_attn_ratio_push), so a layer is two library
+    launches.  The step's buffers are created on the current stream: a step
+    enqueued on another stream must be ordered after them and after the
     inputs (e.g. stream.wait_stream(torch.cuda.current_stream()))."""
 
-    def __init__(self, layers, budget, S, W, n_obs, cu_seqlens=None, max_seqlen=None, group=None):
+    def __init__(self, layers, budget, S, W, n_obs, cu_seqlens=None, max_seqlen=None, group=None, kv_pool=False,
+                 dims=None, fused_push=True):
         if not layers:
             raise ValueError("at least one layer is required")
-        if any(len(lay) != 3 for lay in layers):
+        if any(lay is not None and len(lay) != 3 for lay in layers):
             raise ValueError("every layer must be a (Q, K, V) triple")
+        if any(lay is None for lay in layers) and not kv_pool:
+            raise ValueError("layers given later (None entries) need kv_pool=True")
         if cu_seqlens is not None and max_seqlen is None:
             raise ValueError("max_seqlen is required with cu_seqlens")
-        Q0, K0, _ = layers[0]
-        T, hq, d = Q0.shape
-        hkv = K0.shape[1]
-        for Q, K, V in layers:
-            if Q.shape != Q0.shape or K.shape != K0.shape or V.shape != K0.shape:
+        known = [lay for lay in layers if lay is not None]
+        if dims is None:
+            if not known:
+                raise ValueError("dims=(T, hq, hkv, d) is required when no layer's tensors are given")
+            T, hq, d = known[0][0].shape
+            hkv = known[0][1].shape[1]
+        else:
+            T, hq, hkv, d = (int(x) for x in dims)
+        for Q, K, V in known:
+            if tuple(Q.shape) != (T, hq, d) or tuple(K.shape) != (T, hkv, d) or V.shape != K.shape:
                 raise ValueError("every layer must have the same Q/K/V shapes")
+        if cu_seqlens is not None:
+            # One host read at set-up: tiles past max_seqlen are never scheduled,
+            # so a max_seqlen below the longest sequence would leave rows unwritten.
+            cu = [int(x) for x in cu_seqlens.cpu()]
+            lens = [b - a for a, b in zip(cu[:-1], cu[1:])]
+            if cu[0] != 0 or cu[-1] != T or min(lens, default=0) < 0:
+                raise ValueError("cu_seqlens must rise from 0 to the token count")
+            if int(max_seqlen) < max(lens, default=0):
+                raise ValueError(f"max_seqlen {max_seqlen} is below the longest sequence ({max(lens)})")
         self.layers = list(layers)
         self.L, self.budget, self.S, self.W, self.n_obs = len(layers), int(budget), int(S), int(W), int(n_obs)
+        if not 0 <= self.budget <= self.L:
+            raise ValueError("budget must lie in [0, L]")
         self.T, self.hq, self.hkv, self.d = T, hq, hkv, d
         self.group = group
+        self.kv_pool = bool(kv_pool)
+        # The queue push rides on the attention kernel (its last CTA) unless
+        # the heads are split (the push then follows the ratio exchange) or
+        # fused_push=False (a separate push launch, e.g. to compare the two).
+        self.fused_push = bool(fused_push) and group is None
         self.world = torch.distributed.get_world_size(group) if group is not None else 1
         self.batch = cu_seqlens.numel() - 1 if cu_seqlens is not None else 1
-        dev = Q0.device
+        dev = known[0][0].device if known else torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
         self.kw = dict(cu_seqlens=cu_seqlens, max_seqlen=max_seqlen if cu_seqlens is not None else None)
         self.O = torch.empty((T, hq, d), dtype=torch.bfloat16, device=dev)
         self.LSE = torch.empty((hq, T), dtype=torch.float32, device=dev)
@@ -141,31 +187,60 @@ class PrefillStep:
         self.K_pool = torch.zeros(pool, dtype=torch.bfloat16, device=dev)
         self.V_pool = torch.zeros_like(self.K_pool)
         self.pool_len = torch.zeros((self.budget, self.batch), dtype=torch.int32, device=dev)
-        self.Kp = _b.layer_pointer_table([lay[1] for lay in self.layers], device=dev)
-        self.Vp = _b.layer_pointer_table([lay[2] for lay in self.layers], device=dev)
+        if self.kv_pool:
+            full = (self.L - self.budget, T, hkv, d)
+            self.K_full = torch.empty(full, dtype=torch.bfloat16, device=dev)
+            self.V_full = torch.empty_like(self.K_full)
+            self.Kp = self.Vp = None
+        else:
+            self.K_full = self.V_full = None
+            self.Kp = _b.layer_pointer_table([lay[1] for lay in self.layers], device=dev)
+            self.Vp = _b.layer_pointer_table([lay[2] for lay in self.layers], device=dev)
         self.dq = _b.DeviceQueue(self.L, self.budget, self.batch, device=dev)
 
-    def layer(self, l, stream, O=None, LSE=None, events=None):
-        """Attention + ratio, ratio exchange (sharded), queue push and compaction
-        of layer l; O / LSE default to the step's own scratch."""
-        Q, K, V = self.layers[l]
+    def kv_bytes(self):
+        """(full-KV bytes of one layer, streaming-KV bytes of one demoted layer,
+        bytes the step holds for the KV cache: the full-KV slots, or none when
+        the caller keeps every layer, plus the streaming pool)."""
+        per_row = self.hkv * self.d * 2 * 2       # K and V, bf16
+        full = self.T * per_row
+        stream = self.batch * (self.S + self.W) * per_row
+        held = self.budget * stream + ((self.L - self.budget) * full if self.kv_pool else 0)
+        return full, stream, held
+
+    def layer(self, l, stream, O=None, LSE=None, events=None, qkv=None):
+        """Attention + ratio + queue push, ratio exchange (sharded), and the
+        compaction / slot store of layer l; O / LSE default to the step's own
+        scratch.  qkv: this layer's (Q, K, V), instead of the registered ones
+        (kv_pool mode only)."""
+        if qkv is not None and not self.kv_pool:
+            raise ValueError("qkv= needs kv_pool=True (the registered K/V feed the compaction)")
+        Q, K, V = qkv if qkv is not None else self.layers[l]
+        out = self.O if O is None else O
+        lse = self.LSE if LSE is None else LSE
         if events is not None:
             e0 = torch.cuda.Event(enable_timing=True, external=True)
             e1 = torch.cuda.Event(enable_timing=True, external=True)
             e0.record(stream)
-        _b.lt_prefill_attn_ratio(Q, K, V, self.S, self.W, self.n_obs, out=self.O if O is None else O,
-                                 lse=self.LSE if LSE is None else LSE, ratio=self.ratio[l], stream=stream,
-                                 accumulate=True, **self.kw)
+        if self.fused_push:
+            _b.lt_prefill_attn_ratio_push(Q, K, V, self.S, self.W, self.n_obs, self.dq, l, self.ratio[l], out=out,
+                                          lse=lse, stream=stream, **self.kw)
+        else:
+            _b.lt_prefill_attn_ratio(Q, K, V, self.S, self.W, self.n_obs, out=out, lse=lse, ratio=self.ratio[l],
+                                     stream=stream, accumulate=True, **self.kw)
         if events is not None:
             e1.record(stream)
             events.append((e0, e1))
-        if self.gathered is None:
-            _b.lt_dqueue_push(self.dq.state, self.L, self.batch, l, self.ratio[l], stream)
-        else:
+        if self.gathered is not None:
             with torch.cuda.stream(stream):
                 gather_ratios(self.ratio[l], self.gathered[l], self.group)
             _b.lt_dqueue_push_gathered(self.dq.state, self.L, self.batch, l, self.gathered[l], stream)
-        if self.budget > 0:   # with budget 0 no layer is ever demoted
+        elif not self.fused_push:
+            _b.lt_dqueue_push(self.dq.state, self.L, self.batch, l, self.ratio[l], stream)
+        if self.kv_pool:
+            _b.lt_kv_pool_commit(K, V, self.dq, l, self.S, self.W, self.K_full, self.V_full, self.K_pool,
+                                 self.V_pool, self.pool_len, stream=stream, **self.kw)
+        elif self.budget > 0:   # with budget 0 no layer is ever demoted
             _b.lt_compact_kv_pending(self.Kp, self.Vp, self.dq, self.S, self.W, self.K_pool, self.V_pool,
                                      self.pool_len, self.T, self.hkv, self.d, stream=stream, **self.kw)
 
@@ -186,8 +261,29 @@ class PrefillStep:
         """[L, batch, Hq] ratios of all query heads (this rank's alone when not sharded)."""
         return self.ratio if self.gathered is None else head_ratios(self.gathered)
 
+    def kept_layer_cache(self, l, slots=None):
+        """Full K/V of a layer the queue kept, for lt_decode_attn: (K, V,
+        seq_start) with sequence b's rows starting at row seq_start[b].  In
+        kv_pool mode K/V are the slot pool viewed as [(L - budget) T, hkv, d]
+        and seq_start = slot * T + cu_seqlens[b] (slots: the queue's slot
+        table, read here when not given); otherwise the layer's own tensors."""
+        cu = self.kw["cu_seqlens"]
+        starts = (cu[:-1] if cu is not None else torch.zeros(1, dtype=torch.int32, device=self.device))
+        if not self.kv_pool:
+            _, K, V = self.layers[l]
+            return K, V, starts.to(torch.int32).contiguous()
+        slots = self.dq.slots() if slots is None else slots
+        s = slots[:, l].to(torch.int64)
+        if bool((s < 0).any()):
+            raise ValueError(f"layer {l} holds no full-KV slot (demoted, or not pushed) in some sequence")
+        rows = (self.L - self.budget) * self.T
+        seq_start = (s * self.T + starts.to(torch.int64)).to(torch.int32).contiguous()
+        return (self.K_full.view(rows, self.hkv, self.d), self.V_full.view(rows, self.hkv, self.d), seq_start)
+
     def kernel_launches(self) -> int:
-        """Library kernels one step launches: the queue reset, then attention,
-        push and compaction per layer (the ratio zeroing and the all-gather
-        are torch / NCCL work)."""
-        return 1 + (3 if self.budget > 0 else 2) * self.L
+        """Library kernels one step launches: the queue reset, then per layer
+        the attention (with the queue push when not sharded), the push (when
+        sharded) and the compaction or the slot commit (the ratio zeroing and
+        the all-gather are torch / NCCL work)."""
+        per_layer = 1 + (0 if self.fused_push else 1) + (1 if self.kv_pool or self.budget > 0 else 0)
+        return 1 + per_layer * self.L

@@ -86,10 +86,11 @@ def test_lazy_ratio_rejects_bad_window(S, W, n_obs):
     assert rc == lt.LT_ERR_INVALID_ARG
 
 
-def test_lazy_ratio_rejects_huge_group():
-    s = _shape(hq=128, hkv=1)
+def test_lazy_ratio_rejects_grids_beyond_the_launch_limits():
+    # one CTA cluster per (sequence, query head): hq and batch index grid dimensions of at most 65535
+    s = _shape(hq=70000, hkv=1)
     assert lt.library().lt_lazy_ratio(ctypes.byref(s), FAKE, FAKE, FAKE, 0.0, 4, 32, 16, FAKE, None) == \
-        lt.LT_ERR_UNSUPPORTED
+        lt.LT_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("S,W", [(0, 0), (-1, 3), (2, -1)])
@@ -125,13 +126,16 @@ def test_select_layers_matches_oracle():
                 assert abs(scores[b] - [lt.lt_layer_score(ratios[l, b]) for l in range(L)]).max() < 1e-6
 
 
-def test_select_layers_rejects_nan_and_bad_budget():
+def test_select_layers_rejects_non_finite_scores_and_bad_budget():
     r = np.ones((4, 1, 2), np.float32)
     with pytest.raises(lt.LtError):
         lt.lt_select_layers(r, 5)
-    r[2, 0, 1] = np.nan
-    with pytest.raises(lt.LtError):
-        lt.lt_select_layers(r, 2)
+    # NaN and +-inf are rejected, as the host and device queues reject them.
+    for bad in (np.nan, np.inf, -np.inf):
+        r = np.ones((4, 1, 2), np.float32)
+        r[2, 0, 1] = bad
+        with pytest.raises(lt.LtError):
+            lt.lt_select_layers(r, 2)
 
 
 def test_queue_matches_oracle_every_push_order():

@@ -90,3 +90,22 @@ def test_kv_fraction_after_prefill():
     # budget 0: nothing demoted
     empty = torch.zeros((2, 0), dtype=torch.int32)
     assert bench.kv_fraction_after_prefill(empty, torch.zeros((0, 2), dtype=torch.int32), (5, 7), 3) == 1.0
+
+
+def test_peak_choice_follows_the_averaging_region():
+    """A per-launch time averaged over a short region is held against the
+    burst tensor peak, one averaged over seconds against the sustained one."""
+    peaks = {"bf16_tflops": 1679.2, "bf16_tflops_sustained": 1384.7, "hbm_gbs": 6455.9}
+    peak, why = bench.choose_peak(peaks, 0.004)
+    assert peak == 1679.2 and "burst" in why
+    peak, why = bench.choose_peak(peaks, 5.0)
+    assert peak == 1384.7 and "sustained" in why
+
+
+def test_both_arms_describe_the_workload_alike():
+    cfg = synth.CONFIGS["long128k"]
+    a = bench.workload_config(cfg, True, 1, "replicas")
+    b = bench.workload_config(cfg, True, 1, "replicas")
+    assert a == b and a["kv_pool"] is True and "peak-memory cap" in a["workload"]
+    assert a["parallelism"] == "single GPU"
+    assert bench.workload_config(cfg, True, 2, "heads")["parallelism"].startswith("heads split over 2")

@@ -32,7 +32,7 @@ def exp2_fma(x):
     p = (np.float64(c3) * f.astype(np.float64) + np.float64(c2)).astype(np.float32)
     p = (p.astype(np.float64) * f.astype(np.float64) + np.float64(c1)).astype(np.float32)
     p = (p.astype(np.float64) * f.astype(np.float64) + np.float64(c0)).astype(np.float32)
-    bits = p.view(np.int32).astype(np.int64) + (t.view(np.int32).astype(np.int64) << 23)
+    bits = p.view(np.uint32).astype(np.uint64) + (t.view(np.uint32).astype(np.uint64) << np.uint64(23))
     return (bits & 0xFFFFFFFF).astype(np.uint32).view(np.float32)
 
 

@@ -94,15 +94,15 @@ def test_attention_empty_batch_is_a_no_op():
 @pytest.mark.parametrize("name,n_random", [("gqa1p2b", 400), ("qwen32b", 64), ("batched", 64), ("long128k", 24)])
 def test_attention_full_size_sampled_rows(name, n_random):
     """One layer at the workload's full size, in the launch configuration the
-    benchmark times; the oracle checks sampled rows (the last 128 rows of every
-    sequence for 4 heads, first rows, random rows)."""
+    benchmark times; the oracle checks sampled rows: every observed row (the
+    last max(n_obs, 128) rows of every sequence, a ragged q-tile) of every
+    head, the first rows, and random rows."""
     cfg = synth.CONFIGS[name]
     layer = 1
     Q, K, V = synth.layer_inputs(cfg, layer, "cuda")
     O, LSE = gpu_attention(cfg, Q, K, V)
     torch.cuda.synchronize()
-    last = 128 if name != "long128k" else 32
-    tokens, heads = sample_rows(cfg, n_random, seed=5, last_rows=last, heads_for_last=4 if name != "long128k" else 2)
+    tokens, heads = sample_rows(cfg, n_random, seed=5, last_rows=max(cfg.n_obs, 128), heads_for_last=cfg.hq)
     rel, lse_err = check_attention(cfg, Q, K, V, O, LSE, tokens, heads)
     assert rel <= O_REL_L2 and lse_err <= LSE_ABS, (rel, lse_err)
     assert torch.isfinite(LSE).all() and torch.isfinite(O.float()).all()
@@ -165,21 +165,21 @@ def test_lazy_ratio_closed_forms():
     assert np.abs(r2.cpu().numpy() - 1.0).max() <= RATIO_ABS
 
 
-@pytest.mark.parametrize("name", ["gqa1p2b", "qwen32b", "batched"])
+@pytest.mark.parametrize("name", ["gqa1p2b", "qwen32b", "batched", "long128k"])
 def test_lazy_ratio_full_size(name):
-    """Full size: the ratio kernel against the oracle given the same LSE (the
-    oracle's own LSE costs a full prefill per observed row at these sizes; the
-    LSE of the observed rows is checked against the oracle in the attention
-    tests), and for gqa1p2b also end to end against the oracle's own LSE."""
+    """Full size, in the launch configuration the benchmark times: the ratio
+    kernel end to end (its LSE from the GPU attention) against the oracle with
+    its own LSE (one full attention row per observed row and head), and as a
+    unit against the oracle given the same LSE."""
     cfg = synth.CONFIGS[name]
     Q, K, V = synth.layer_inputs(cfg, 2, "cuda")
     _, LSE = gpu_attention(cfg, Q, K, V)
     r = gpu_ratio(cfg, Q, K, LSE)
     torch.cuda.synchronize()
+    got = r.cpu().numpy()
+    assert np.abs(got - oracle_ratio(cfg, Q, K)).max() <= RATIO_ABS
     ref = oracle_ratio(cfg, Q, K, lse=LSE.cpu().numpy().astype(np.float64))
-    assert np.abs(r.cpu().numpy() - ref).max() <= RATIO_ABS
-    if name == "gqa1p2b":
-        assert np.abs(r.cpu().numpy() - oracle_ratio(cfg, Q, K)).max() <= RATIO_ABS
+    assert np.abs(got - ref).max() <= RATIO_ABS
     del Q, K, V, LSE
     torch.cuda.empty_cache()
 
@@ -295,15 +295,22 @@ def test_fused_attention_ratio(spec):
         assert np.abs(r.cpu().numpy() - r_sep.cpu().numpy()).max() <= 1e-4
 
 
-@pytest.mark.parametrize("name", ["gqa1p2b", "qwen32b"])
+@pytest.mark.parametrize("name", ["gqa1p2b", "qwen32b", "batched", "long128k"])
 def test_fused_ratio_full_size(name):
+    """The fused ratio at full size against the oracle with its own LSE (end to
+    end), against the oracle given the kernel's LSE, and against the separate
+    pass."""
     cfg = synth.CONFIGS[name]
     from tests.gpu_common import gpu_fused
     Q, K, V = synth.layer_inputs(cfg, 3, "cuda")
     O, LSE, r = gpu_fused(cfg, Q, K, V)
     r2 = gpu_ratio(cfg, Q, K, LSE)
+    O1, L1 = gpu_attention(cfg, Q, K, V)
     torch.cuda.synchronize()
+    assert torch.equal(O, O1) and torch.equal(LSE, L1)     # the plain kernel's O and LSE, bit for bit
+    del O1, L1
     assert np.abs(r.cpu().numpy() - r2.cpu().numpy()).max() <= 1e-4
+    assert np.abs(r.cpu().numpy() - oracle_ratio(cfg, Q, K)).max() <= RATIO_ABS
     ref = oracle_ratio(cfg, Q, K, lse=LSE.cpu().numpy().astype(np.float64))
     assert np.abs(r.cpu().numpy() - ref).max() <= RATIO_ABS
     # Run-to-run reproducibility of the fused ratio (n_obs <= 128).
