@@ -424,28 +424,40 @@ def run_ours(args, cfg, rank, world):
     # layer (all layers twice for short steps, the first four once for long ones).
     kw = pf.kw
     side_layers = list(range(min(cfg.layers, 4))) if long_step else list(range(cfg.layers))
-    attn_ev, ratio_ev = [], []
+    # The fused kernel is timed in the same loop (its zeroing form), right after
+    # the plain one on the same inputs, so the ratio's overhead compares the
+    # two kernels under the same conditions (clock, power, L2).
+    attn_ev, ratio_ev, fused_eager_ev = [], [], []
     ratio_out = torch.empty_like(pf.ratio[0])
     for rep in range(2 if not long_step else 1):
         for l in side_layers:
             Q, K, V = pf.layers[l]
-            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0, e1, e2, e3 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
             e0.record()
             lt.lt_prefill_attn(Q, K, V, out=pf.O, lse=pf.LSE, **kw)
             e1.record()
             lt.lt_lazy_ratio(Q, K, pf.LSE, cfg.S, cfg.W, cfg.n_obs, out=ratio_out, **kw)
-            e2.record()
+            ratio_out.zero_()      # outside the fused launch's events (accumulate form, as in the step)
+            e2b = torch.cuda.Event(enable_timing=True)
+            e2b.record()
+            lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, out=pf.O, lse=pf.LSE, ratio=ratio_out,
+                                     accumulate=True, **kw)
+            e3.record()
             if rep > 0 or long_step and l > 0:
                 attn_ev.append((e0, e1))
                 ratio_ev.append((e1, e2))
+                fused_eager_ev.append((e2b, e3))
     torch.cuda.synchronize()
     t_attn = statistics.mean(a.elapsed_time(b) for a, b in attn_ev) * 1e-3
     t_ratio = statistics.mean(a.elapsed_time(b) for a, b in ratio_ev) * 1e-3
+    t_fused_eager = statistics.mean(a.elapsed_time(b) for a, b in fused_eager_ev) * 1e-3
     kv = pf.kv_report(step_alloc)
 
     if args.kernels_only:
         return {"metric": METRIC, "config": {"workload": cfg.name, "kv_pool": kv_pool},
                 "ms_per_step": round(ms, 4), "fused_us_per_layer": round(t_fused * 1e6, 2),
+                "fused_eager_us_per_layer": round(t_fused_eager * 1e6, 2),
+                "fused_ratio_overhead_pct": round(100 * (t_fused_eager - t_attn) / t_attn, 3),
                 "attn_us_per_layer": round(t_attn * 1e6, 2), "ratio_us_per_layer": round(t_ratio * 1e6, 2),
                 "kv_cache_fraction_after_prefill": round(kv_frac, 4), "kv_cache": kv, "gpu_launches": launches,
                 "events_region_s": round(events_region_s, 3)}
@@ -525,10 +537,11 @@ def run_ours(args, cfg, rank, world):
         "config": workload_config(cfg, kv_pool, world, args.shard),
         "attn_tflops": round(achieved, 2),
         "attn_pct_of_burst_peak": round(100 * achieved / peak_burst, 2),
-        "fused_attn_ratio_us_per_layer": round(t_fused * 1e6, 2),
+        "fused_attn_ratio_push_us_per_layer_in_step": round(t_fused * 1e6, 2),
+        "fused_attn_ratio_us_per_layer": round(t_fused_eager * 1e6, 2),
         "attn_only_us_per_layer": round(t_attn * 1e6, 2),
         "attn_only_tflops": round(fl_attn / t_attn / 1e12, 2),
-        "fused_ratio_overhead_pct": round(100 * (t_fused - t_attn) / t_attn, 3),
+        "fused_ratio_overhead_pct": round(100 * (t_fused_eager - t_attn) / t_attn, 3),
         "separate_ratio_us_per_layer": round(t_ratio * 1e6, 2),
         "separate_ratio_overhead_pct": round(100 * t_ratio / t_attn, 3),
         "compaction_gbs": round(comp_gbs, 1),
@@ -583,9 +596,23 @@ def measure_decode(cfg, lt, pf, peaks):
         K, V, st = pf.step.kept_layer_cache(l, slots)
         full_cache[l] = (K, V, st if pf.kv_pool else starts)
 
-    def full(l, s):
+    workspace = torch.empty(max(16, lt.lt_decode_splitk_workspace_bytes(B, cfg.hq, d, cfg.max_seqlen)),
+                            dtype=torch.uint8, device="cuda")
+
+    def full_cluster(l, s):
         K, V, st = full_cache[l] if l in full_cache else (pf.layers[l][1], pf.layers[l][2], starts)
         lt.lt_decode_attn(q, K, V, lens, seq_start=st, max_len=cfg.max_seqlen, out=O, lse=LSE, stream=s)
+
+    def full_splitk(l, s):
+        K, V, st = full_cache[l] if l in full_cache else (pf.layers[l][1], pf.layers[l][2], starts)
+        lt.lt_decode_attn_splitk(q, K, V, lens, seq_start=st, max_len=cfg.max_seqlen, out=O, lse=LSE,
+                                 workspace=workspace, stream=s)
+
+    full_paths = {"cluster": full_cluster, "splitk": full_splitk}
+    choice = {"path": "cluster"}
+
+    def full(l, s):
+        full_paths[choice["path"]](l, s)
 
     def streaming(l, s):
         k = slot_of[l]
@@ -622,13 +649,21 @@ def measure_decode(cfg, lt, pf, peaks):
                 out.append(e0.elapsed_time(e1) * 1e-3)
         return statistics.median(out)
 
+    l0 = min(full_cache) if full_cache else 0
+    t_path = {name: timed(lambda s, fn=fn: fn(l0, s), reps=20) for name, fn in full_paths.items()}
+    choice["path"] = min(t_path, key=t_path.get)       # the faster full-cache decode for this length
     t_hybrid = timed(hybrid_step)
     t_full = timed(full_step)
-    t_full_layer = timed(lambda s: full(min(full_cache) if full_cache else 0, s), reps=20)
+    t_full_layer = t_path[choice["path"]]
     t_stream_layer = timed(lambda s: streaming(demoted[0], s), reps=20) if demoted else None
     del flush
     n_rows = sum(cu_h[b + 1] - cu_h[b] for b in range(B))
     full_bytes = n_rows * cfg.hkv * d * 2 * 2 + 2 * B * cfg.hq * d * 2 + B * cfg.hq * 4
+    # K/V bytes a decode token reads: every layer full, or the demoted ones on
+    # their streaming caches (the ratio the hybrid speed-up tends to when HBM bound).
+    stream_rows = sum(min(cu_h[b + 1] - cu_h[b], cfg.S + cfg.W) for b in range(B))
+    full_step_bytes = cfg.layers * n_rows * cfg.hkv * d * 4
+    hybrid_step_bytes = ((cfg.layers - len(demoted)) * n_rows + len(demoted) * stream_rows) * cfg.hkv * d * 4
     peak_hbm = float(peaks["hbm_gbs"])
     gbs = full_bytes / t_full_layer / 1e9
     out = {
@@ -639,6 +674,9 @@ def measure_decode(cfg, lt, pf, peaks):
         "decode_full_layer_us": round(t_full_layer * 1e6, 2),
         "decode_full_layer_gbs": round(gbs, 1),
         "decode_full_layer_frac_of_hbm": round(gbs / peak_hbm, 4),
+        "decode_full_layer_path": choice["path"],
+        "decode_full_layer_us_by_path": {k: round(v * 1e6, 2) for k, v in t_path.items()},
+        "decode_speedup_analytic_bytes": round(full_step_bytes / hybrid_step_bytes, 3),
     }
     if t_stream_layer is not None:
         slots = cfg.S + cfg.W

@@ -386,6 +386,28 @@ lt_status lt_decode_attn(const void* q, const void* K, const void* V, const int3
                          float* LSE, float softmax_scale, lt_stream stream);
 
 /*
+ * lt_decode_attn for long caches: the same decode step (same arguments,
+ * layouts, results and errors, except head_dim 64/128 and the workspace),
+ * with the rows of each (sequence, KV head) split over
+ * ceil(max_len / 1024) CTAs (at most 128; any number, where lt_decode_attn's
+ * cluster split stops at 16), so that a batch-1 decode over a few KV heads
+ * keeps every SM streaming K/V.  Each CTA writes its partial softmax state
+ * (running max and sum, unnormalised output of every query head) to
+ * `workspace`; a second kernel merges the splits of each head in split order
+ * (deterministic).  workspace: caller-allocated device memory of at least
+ * lt_decode_splitk_workspace_bytes(batch, hq, head_dim, max_len) bytes
+ * (batch * hq * splits * (head_dim + 2) floats), 16-byte aligned; its
+ * contents on entry do not matter and on return are scratch.  Two launches on
+ * `stream`; calls that share a workspace must not overlap.
+ * LT_ERR_INVALID_ARG also for a missing or too small workspace.
+ */
+size_t lt_decode_splitk_workspace_bytes(int batch, int hq, int head_dim, int max_len);
+lt_status lt_decode_attn_splitk(const void* q, const void* K, const void* V, const int32_t* seq_start,
+                                int seq_capacity, const int32_t* len, int batch, int hq, int hkv, int head_dim,
+                                int max_len, void* O, float* LSE, float softmax_scale, void* workspace,
+                                size_t workspace_bytes, lt_stream stream);
+
+/*
  * Device status word of the current device: LT_OK, or LT_ERR_TIMEOUT if a kernel
  * gave up a bounded wait since the last clear.  Synchronises the device.
  * clear != 0 resets the word.

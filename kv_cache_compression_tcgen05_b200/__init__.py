@@ -52,6 +52,8 @@ from .binding import (  # noqa: F401
     lt_stream_append,
     lt_stream_decode,
     lt_decode_attn,
+    lt_decode_attn_splitk,
+    lt_decode_splitk_workspace_bytes,
     lt_stream_ring_init,
 )
 from .build import build  # noqa: F401

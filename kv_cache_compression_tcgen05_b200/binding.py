@@ -71,6 +71,9 @@ _SIGS = {
     "lt_stream_append": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp]),
     "lt_stream_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp]),
     "lt_decode_attn": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp]),
+    "lt_decode_splitk_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i]),
+    "lt_decode_attn_splitk": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp,
+                                   ctypes.c_size_t, _vp]),
     "lt_device_status": (_i, [_i]),
     "lt_selftest_wait_timeout": (_i, [ctypes.c_uint, _vp]),
     "lt_status_string": (ctypes.c_char_p, [_i]),
@@ -602,13 +605,10 @@ def lt_stream_decode(q, K_stream, V_stream, stream_len, softmax_scale=None, out=
     return out, lse
 
 
-def lt_decode_attn(q, K, V, seq_len, seq_start=None, max_len=None, softmax_scale=None, out=None, lse=None,
-                   stream=None):
-    """Decode attention over a kept layer's full cache: q [batch, hq, d] ->
-    (O [batch, hq, d], LSE [batch, hq]).  K/V either token-major packed
-    [rows, hkv, d] with seq_start (device int32 [batch], first row of each
-    sequence), or padded [batch, capacity, hkv, d] with seq_start None.
-    seq_len: device int32 [batch] positions attended."""
+def _decode_full_args(q, K, V, seq_len, seq_start, max_len, out, lse):
+    """Checked arguments of a decode over a full cache (shared by the cluster
+    and split-K calls): (q, K, V, seq_start, capacity, len, B, hq, hkv, d,
+    max_len, out, lse)."""
     _dev_tensor(q, "q", torch.bfloat16, 3)
     B, hq, d = q.shape
     if K.dim() == 4:
@@ -640,9 +640,45 @@ def lt_decode_attn(q, K, V, seq_len, seq_start=None, max_len=None, softmax_scale
         lse = torch.empty((B, hq), dtype=torch.float32, device=q.device)
     _sized(out, "out", torch.bfloat16, (B, hq, d))
     _sized(lse, "lse", torch.float32, (B, hq))
+    return q, K, V, seq_start, cap, seq_len, B, hq, hkv, d, limit, out, lse
+
+
+def lt_decode_attn(q, K, V, seq_len, seq_start=None, max_len=None, softmax_scale=None, out=None, lse=None,
+                   stream=None):
+    """Decode attention over a kept layer's full cache: q [batch, hq, d] ->
+    (O [batch, hq, d], LSE [batch, hq]).  K/V either token-major packed
+    [rows, hkv, d] with seq_start (device int32 [batch], first row of each
+    sequence), or padded [batch, capacity, hkv, d] with seq_start None.
+    seq_len: device int32 [batch] positions attended."""
+    q, K, V, seq_start, cap, seq_len, B, hq, hkv, d, limit, out, lse = _decode_full_args(
+        q, K, V, seq_len, seq_start, max_len, out, lse)
     _check(library().lt_decode_attn(q.data_ptr(), K.data_ptr(), V.data_ptr(),
                                     None if seq_start is None else seq_start.data_ptr(), cap, seq_len.data_ptr(), B,
                                     hq, hkv, d, limit, out.data_ptr(), lse.data_ptr(),
                                     0.0 if softmax_scale is None else float(softmax_scale), _stream_handle(stream)),
            "lt_decode_attn")
+    return out, lse
+
+
+def lt_decode_splitk_workspace_bytes(batch, hq, head_dim, max_len) -> int:
+    return int(library().lt_decode_splitk_workspace_bytes(int(batch), int(hq), int(head_dim), int(max_len)))
+
+
+def lt_decode_attn_splitk(q, K, V, seq_len, seq_start=None, max_len=None, softmax_scale=None, out=None, lse=None,
+                          workspace=None, stream=None):
+    """lt_decode_attn for long caches, split over many CTAs with a workspace
+    (device uint8 tensor of at least lt_decode_splitk_workspace_bytes bytes;
+    allocated here when None).  Same arguments and results otherwise."""
+    q, K, V, seq_start, cap, seq_len, B, hq, hkv, d, limit, out, lse = _decode_full_args(
+        q, K, V, seq_len, seq_start, max_len, out, lse)
+    need = lt_decode_splitk_workspace_bytes(B, hq, d, limit)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _dev_tensor(workspace, "workspace", torch.uint8, 1)
+    _check(library().lt_decode_attn_splitk(q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                           None if seq_start is None else seq_start.data_ptr(), cap,
+                                           seq_len.data_ptr(), B, hq, hkv, d, limit, out.data_ptr(), lse.data_ptr(),
+                                           0.0 if softmax_scale is None else float(softmax_scale),
+                                           workspace.data_ptr(), workspace.numel(), _stream_handle(stream)),
+           "lt_decode_attn_splitk")
     return out, lse

@@ -92,9 +92,17 @@ struct AttnLayout {
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 64;
   static constexpr int kAlloc = kBytes + 1024;        // room to align the base to 1024 B
-  // 10 working warps; two more idle warps make ptxas allocate the softmax
-  // path without spills (same 168 registers per thread either way).
+  // Three warpgroups: softmax of tile A (warps 0..3) and of tile B (4..7),
+  // and a third holding the TMA producer (warp 8), the TMEM owner / MMA
+  // issuer (warp 9) and two idle warps.  Launched at 168 registers a thread
+  // (one CTA per SM); setmaxnreg then moves registers from the third
+  // warpgroup to the softmax ones.
   static constexpr int kThreads = 384;
+  static constexpr int kLaunchRegs = 168;
+  static constexpr int kRegsSoftmax = 184;
+  static constexpr int kRegsOther = 3 * kLaunchRegs - 2 * kRegsSoftmax;   // 136
+  static constexpr int kWarpProducer = 8;
+  static constexpr int kWarpMma = 9;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmemO = 256;
 };
@@ -195,6 +203,7 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int grid = gridDim.x;
   const int cta = blockIdx.x;
+  constexpr int kWarpProducer = Lay::kWarpProducer, kWarpMma = Lay::kWarpMma;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -218,7 +227,7 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_slot, Lay::kTmemCols);
     tmem_relinquish();
   }
@@ -232,133 +241,142 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitCtl ctl{abort_flag, p.status};
   const WaitCtl drain_ctl{no_abort, p.status};
-  if (warp == 0) {
-    // ------------------------------------------------------------- producer
-    if (lane == 0) {
-      int ring = 0, nq = 0;
-      bool ok = true;
-      for (int round = 0; ok && round * grid < p.num_items; ++round) {
-        const int t = attn_item_index(round, cta, grid);
-        AttnItem it;
-        if (t >= p.num_items || !attn_decode(p, t, it)) continue;
-        const int qb = nq & 1;
-        if (nq >= 2 && !(ok = mbar_wait(&q_empty[qb], ((nq >> 1) - 1) & 1, ctl))) break;
-        const int ntile = it.hasB ? 2 : 1;
-        mbar_expect_tx(&q_full[qb], ntile * Lay::kTileBytes);
-        for (int x = 0; x < ntile; ++x)
-          for (int st = 0; st < D / 64; ++st)
-            tma_load_3d(sQ + (qb * 2 + x) * Lay::kTileBytes + st * Lay::kSub, &tmQ, &q_full[qb], st * 64, it.h[x],
-                        it.start + it.qt[x] * 128);
-        ++nq;
-        // Ring order: K0, V0, K1, V1, ...
-        for (int j = 0; ok && j < it.n[0]; ++j) {
-          for (int kv = 0; kv < 2; ++kv) {
-            const int slot = ring % Lay::kStages;
-            if (ring >= Lay::kStages && !(ok = mbar_wait(&kv_empty[slot], ((ring / Lay::kStages) - 1) & 1, ctl)))
-              break;
-            mbar_expect_tx(&kv_full[slot], Lay::kTileBytes);
+  // Role dispatch by warpgroup: setmaxnreg is executed by all four warps of
+  // a warpgroup at the start of its branch, so each branch is compiled under
+  // its own register limit.  2 * kRegsSoftmax + kRegsOther = 3 * the
+  // launch's 168 registers a thread (checked on the host against the
+  // compiled kernel before any launch).
+  if (warp >= 8) {
+    regs_decrease<Lay::kRegsOther>();
+    if (warp == kWarpProducer) {
+      // ------------------------------------------------------------- producer
+      if (lane == 0) {
+        int ring = 0, nq = 0;
+        bool ok = true;
+        for (int round = 0; ok && round * grid < p.num_items; ++round) {
+          const int t = attn_item_index(round, cta, grid);
+          AttnItem it;
+          if (t >= p.num_items || !attn_decode(p, t, it)) continue;
+          const int qb = nq & 1;
+          if (nq >= 2 && !(ok = mbar_wait(&q_empty[qb], ((nq >> 1) - 1) & 1, ctl))) break;
+          const int ntile = it.hasB ? 2 : 1;
+          mbar_expect_tx(&q_full[qb], ntile * Lay::kTileBytes);
+          for (int x = 0; x < ntile; ++x)
             for (int st = 0; st < D / 64; ++st)
-              tma_load_3d(sRing + slot * Lay::kTileBytes + st * Lay::kSub, kv == 0 ? &tmK : &tmV, &kv_full[slot],
-                          st * 64, it.kh, it.start + j * 128);
-            ++ring;
+              tma_load_3d(sQ + (qb * 2 + x) * Lay::kTileBytes + st * Lay::kSub, &tmQ, &q_full[qb], st * 64, it.h[x],
+                          it.start + it.qt[x] * 128);
+          ++nq;
+          // Ring order: K0, V0, K1, V1, ...
+          for (int j = 0; ok && j < it.n[0]; ++j) {
+            for (int kv = 0; kv < 2; ++kv) {
+              const int slot = ring % Lay::kStages;
+              if (ring >= Lay::kStages && !(ok = mbar_wait(&kv_empty[slot], ((ring / Lay::kStages) - 1) & 1, ctl)))
+                break;
+              mbar_expect_tx(&kv_full[slot], Lay::kTileBytes);
+              for (int st = 0; st < D / 64; ++st)
+                tma_load_3d(sRing + slot * Lay::kTileBytes + st * Lay::kSub, kv == 0 ? &tmK : &tmV, &kv_full[slot],
+                            st * 64, it.kh, it.start + j * 128);
+              ++ring;
+            }
           }
         }
+        if (!ok) {
+          // Let the loads already issued land before the CTA's shared memory is
+          // released (bounded; the abort flag is ignored here).
+          for (int x = ring > Lay::kStages ? ring - Lay::kStages : 0; x < ring; ++x)
+            mbar_wait(&kv_full[x % Lay::kStages], (x / Lay::kStages) & 1, drain_ctl);
+          for (int x = nq > 2 ? nq - 2 : 0; x < nq; ++x) mbar_wait(&q_full[x & 1], (x >> 1) & 1, drain_ctl);
+        }
       }
-      if (!ok) {
-        // Let the loads already issued land before the CTA's shared memory is
-        // released (bounded; the abort flag is ignored here).
-        for (int x = ring > Lay::kStages ? ring - Lay::kStages : 0; x < ring; ++x)
-          mbar_wait(&kv_full[x % Lay::kStages], (x / Lay::kStages) & 1, drain_ctl);
-        for (int x = nq > 2 ? nq - 2 : 0; x < nq; ++x) mbar_wait(&q_full[x & 1], (x >> 1) & 1, drain_ctl);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------- MMA
-    if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
-      // Shared-memory descriptors differ only in the start-address field
-      // (address / 16, 14 bits; the shared window is below 256 KB): built once,
-      // advanced by byte offset / 16 per MMA.
-      const uint64_t q_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
-      const uint64_t k_desc = smem_desc_sw128(smem_u32(sRing), 16, 1024);
-      const uint64_t v_desc = smem_desc_sw128(smem_u32(sRing), Lay::kSub, 1024);
-      int ring = 0, nq = 0;
-      int cnt_p0 = 0, cnt_p1 = 0;   // P tiles consumed, per tile slot
-      int cnt_o0 = 0, cnt_o1 = 0;   // items finished, per tile slot
-      bool ok = true;
-      for (int round = 0; ok && round * grid < p.num_items; ++round) {
-        const int t = attn_item_index(round, cta, grid);
-        AttnItem it;
-        if (t >= p.num_items || !attn_decode(p, t, it)) continue;
-        const int qb = nq & 1;
-        if (!(ok = mbar_wait(&q_full[qb], (nq >> 1) & 1, ctl))) break;
-        ++nq;
-        const int base = ring;
-        const int n = it.n[0];
-        const int nB = it.hasB ? it.n[1] : 0;
-        ring = base + 2 * n;
-        auto slot_of = [&](int j, int kv) { return (base + 2 * j + kv) % Lay::kStages; };
-        auto phase_of = [&](int j, int kv) { return ((base + 2 * j + kv) / Lay::kStages) & 1; };
-        // S_x(j) = Q_x K_j^T into the tile's TMEM score columns.
-        auto issue_s = [&](int x, int j) -> bool {
-          const int slot = slot_of(j, 0);
-          if (x == 0) {   // tile A always uses K_j first
-            if (!mbar_wait(&kv_full[slot], phase_of(j, 0), ctl)) return false;
-          }
-          tc_fence_after();
-          const uint64_t qd = q_desc + uint64_t(((qb * 2 + x) * Lay::kTileBytes) >> 4);
-          const uint64_t kd = k_desc + uint64_t((slot * Lay::kTileBytes) >> 4);
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off16 = ((k >> 2) * Lay::kSub + (k & 3) * 32) >> 4;
-            mma_bf16_ss(tmem + x * 128, qd + off16, kd + off16, kIdS, k > 0 ? 1u : 0u);
-          }
-          mma_commit(&s_full[x]);
-          const bool last_use = x == 1 || j >= nB;
-          if (last_use) mma_commit(&kv_empty[slot]);
-          if (last_use && j == n - 1) mma_commit(&q_empty[qb]);
-          return true;
-        };
-        // O_x += P_x(j) V_j, P_x(j) read from TMEM.
-        auto issue_pv = [&](int x, int j) -> bool {
-          int& cnt_p = x ? cnt_p1 : cnt_p0;
-          int& cnt_o = x ? cnt_o1 : cnt_o0;
-          if (!mbar_wait(&p_full[x], cnt_p & 1, ctl)) return false;
-          ++cnt_p;
-          if (j == 0 && cnt_o > 0 && !mbar_wait(&o_empty[x], (cnt_o - 1) & 1, ctl)) return false;
-          const int slot = slot_of(j, 1);
-          if (x == 0 && !mbar_wait(&kv_full[slot], phase_of(j, 1), ctl)) return false;
-          tc_fence_after();
-          const uint64_t vd = v_desc + uint64_t((slot * Lay::kTileBytes) >> 4);
-          const uint32_t o_tmem = tmem + Lay::kTmemO + x * D;
-#pragma unroll
-          for (int k = 0; k < 128 / 16; ++k)
-            mma_bf16_ts(o_tmem, tmem + x * 128 + k * 8, vd + uint64_t((k * 2048) >> 4), kIdPV,
-                        (j > 0 || k > 0) ? 1u : 0u);
-          const bool last_use = x == 1 || j >= nB;
-          if (last_use) mma_commit(&kv_empty[slot]);
-          if ((x == 0 && j == n - 1) || (x == 1 && j == nB - 1)) {
-            mma_commit(&o_full[x]);
-            ++cnt_o;
-          }
-          return true;
-        };
+    } else if (warp == kWarpMma) {
+      // ------------------------------------------------------------------- MMA
+      if (lane == 0) {
+        constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
+        // Shared-memory descriptors differ only in the start-address field
+        // (address / 16, 14 bits; the shared window is below 256 KB): built once,
+        // advanced by byte offset / 16 per MMA.
+        const uint64_t q_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+        const uint64_t k_desc = smem_desc_sw128(smem_u32(sRing), 16, 1024);
+        const uint64_t v_desc = smem_desc_sw128(smem_u32(sRing), Lay::kSub, 1024);
+        int ring = 0, nq = 0;
+        int cnt_p0 = 0, cnt_p1 = 0;   // P tiles consumed, per tile slot
+        int cnt_o0 = 0, cnt_o1 = 0;   // items finished, per tile slot
+        bool ok = true;
+        for (int round = 0; ok && round * grid < p.num_items; ++round) {
+          const int t = attn_item_index(round, cta, grid);
+          AttnItem it;
+          if (t >= p.num_items || !attn_decode(p, t, it)) continue;
+          const int qb = nq & 1;
+          if (!(ok = mbar_wait(&q_full[qb], (nq >> 1) & 1, ctl))) break;
+          ++nq;
+          const int base = ring;
+          const int n = it.n[0];
+          const int nB = it.hasB ? it.n[1] : 0;
+          ring = base + 2 * n;
+          auto slot_of = [&](int j, int kv) { return (base + 2 * j + kv) % Lay::kStages; };
+          auto phase_of = [&](int j, int kv) { return ((base + 2 * j + kv) / Lay::kStages) & 1; };
+          // S_x(j) = Q_x K_j^T into the tile's TMEM score columns.
+          auto issue_s = [&](int x, int j) -> bool {
+            const int slot = slot_of(j, 0);
+            if (x == 0) {   // tile A always uses K_j first
+              if (!mbar_wait(&kv_full[slot], phase_of(j, 0), ctl)) return false;
+            }
+            tc_fence_after();
+            const uint64_t qd = q_desc + uint64_t(((qb * 2 + x) * Lay::kTileBytes) >> 4);
+            const uint64_t kd = k_desc + uint64_t((slot * Lay::kTileBytes) >> 4);
+  #pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint32_t off16 = ((k >> 2) * Lay::kSub + (k & 3) * 32) >> 4;
+              mma_bf16_ss(tmem + x * 128, qd + off16, kd + off16, kIdS, k > 0 ? 1u : 0u);
+            }
+            mma_commit(&s_full[x]);
+            const bool last_use = x == 1 || j >= nB;
+            if (last_use) mma_commit(&kv_empty[slot]);
+            if (last_use && j == n - 1) mma_commit(&q_empty[qb]);
+            return true;
+          };
+          // O_x += P_x(j) V_j, P_x(j) read from TMEM.
+          auto issue_pv = [&](int x, int j) -> bool {
+            int& cnt_p = x ? cnt_p1 : cnt_p0;
+            int& cnt_o = x ? cnt_o1 : cnt_o0;
+            if (!mbar_wait(&p_full[x], cnt_p & 1, ctl)) return false;
+            ++cnt_p;
+            if (j == 0 && cnt_o > 0 && !mbar_wait(&o_empty[x], (cnt_o - 1) & 1, ctl)) return false;
+            const int slot = slot_of(j, 1);
+            if (x == 0 && !mbar_wait(&kv_full[slot], phase_of(j, 1), ctl)) return false;
+            tc_fence_after();
+            const uint64_t vd = v_desc + uint64_t((slot * Lay::kTileBytes) >> 4);
+            const uint32_t o_tmem = tmem + Lay::kTmemO + x * D;
+  #pragma unroll
+            for (int k = 0; k < 128 / 16; ++k)
+              mma_bf16_ts(o_tmem, tmem + x * 128 + k * 8, vd + uint64_t((k * 2048) >> 4), kIdPV,
+                          (j > 0 || k > 0) ? 1u : 0u);
+            const bool last_use = x == 1 || j >= nB;
+            if (last_use) mma_commit(&kv_empty[slot]);
+            if ((x == 0 && j == n - 1) || (x == 1 && j == nB - 1)) {
+              mma_commit(&o_full[x]);
+              ++cnt_o;
+            }
+            return true;
+          };
 
-        ok = issue_s(0, 0) && (nB == 0 || issue_s(1, 0));
-        for (int j = 0; ok && j < n; ++j) {
-          ok = issue_pv(0, j) && (j + 1 >= n || issue_s(0, j + 1));
-          if (ok && j < nB) ok = issue_pv(1, j) && (j + 1 >= nB || issue_s(1, j + 1));
+          ok = issue_s(0, 0) && (nB == 0 || issue_s(1, 0));
+          for (int j = 0; ok && j < n; ++j) {
+            ok = issue_pv(0, j) && (j + 1 >= n || issue_s(0, j + 1));
+            if (ok && j < nB) ok = issue_pv(1, j) && (j + 1 >= nB || issue_s(1, j + 1));
+          }
+        }
+        if (!ok) {
+          mma_commit(drain);
+          mbar_wait(drain, 0, drain_ctl);
         }
       }
-      if (!ok) {
-        mma_commit(drain);
-        mbar_wait(drain, 0, drain_ctl);
-      }
     }
-  } else if (warp < 10) {
+  } else {
+    regs_increase<Lay::kRegsSoftmax>();
     // --------------------------------------------------------------- softmax
-    const int x = (warp - 2) >> 2;             // tile slot: 0 = A (warps 2..5), 1 = B (warps 6..9)
+    const int x = warp >> 2;                   // tile slot: 0 = A (warps 0..3), 1 = B (warps 4..7)
     const int wq = warp & 3;                   // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;            // query row within the tile
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
@@ -551,7 +569,7 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, Lay::kTmemCols);
   }

@@ -277,4 +277,222 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
   }
 }
 
+// ----------------------------------------------------------- split-K decode
+//
+// Long caches: the cluster split above puts at most kDecodeMaxSplits CTAs on a
+// (sequence, KV head), so a batch-1 decode over 8 KV heads uses 128 of the
+// 148 SMs with one row in flight per lane group, and is bound by memory
+// latency, not bandwidth.  Here the rows of a (sequence, KV head) are split
+// over `splits` independent CTAs (any number, no cluster), each lane group
+// takes two rows per iteration (both prefetched one iteration ahead, so four
+// 16-byte loads are in flight per lane), and each CTA writes its partial
+// softmax state -- running max and sum in the log2 domain and the unnormalised
+// output of each query head -- to a workspace; decode_merge_kernel then
+// combines the splits of each head in split order.  The workspace is the only
+// memory written beyond the outputs.
+constexpr int kDecodeMaxSplitK = 128;
+constexpr int kDecodeRowsPerSplit = 1024;   // rows of the longest cache per split
+
+// CTAs per (sequence, KV head) of the split-K decode for caches of up to
+// max_len rows (a pure function of max_len, so a caller can size the
+// workspace without the device).
+__host__ __device__ inline int decode_splitk_splits(int max_len) {
+  const int s = (max_len + kDecodeRowsPerSplit - 1) / kDecodeRowsPerSplit;
+  return s < 1 ? 1 : (s > kDecodeMaxSplitK ? kDecodeMaxSplitK : s);
+}
+
+// Floats of split-K workspace: [batch, hq, splits, D + 2] (output, max, sum).
+__host__ __device__ inline size_t decode_splitk_floats(int batch, int hq, int head_dim, int max_len) {
+  return size_t(batch) * hq * decode_splitk_splits(max_len) * (head_dim + 2);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecodeThreads) decode_splitk_kernel(const DecodeParams p, float* part) {
+  constexpr int E = 8;           // elements of a row per lane (one 16-byte load)
+  constexpr int LPR = D / E;     // lanes per row
+  constexpr int GPW = 32 / LPR;  // row groups per warp
+  const int split = blockIdx.x % p.splits;
+  const int kh = blockIdx.x / p.splits;
+  const int b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rgw = lane / LPR;
+  const int li = lane % LPR;
+  __shared__ float sm_m[kDecodeWarps][kDecodeHeads], sm_l[kDecodeWarps][kDecodeHeads];
+  __shared__ __align__(16) float sm_o[kDecodeWarps][kDecodeHeads][D];
+
+  const int n = min(max(p.len[b], 0), p.max_len);
+  const int chunk = (n + p.splits - 1) / p.splits;
+  const int r_begin = min(n, split * chunk);
+  const int r_end = min(n, r_begin + chunk);
+  const long long seq_off = p.seq_start ? (long long)p.seq_start[b] * p.row_stride : (long long)b * p.seq_stride;
+  const __nv_bfloat16* Kb = p.K + seq_off + kh * p.head_stride + li * E;
+  const __nv_bfloat16* Vb = p.V + seq_off + kh * p.head_stride + li * E;
+  constexpr int kRowsPerIter = kDecodeWarps * GPW;   // rows of one sweep of the CTA
+  constexpr int kStep = 2 * kRowsPerIter;             // two sweeps per iteration
+
+  auto unpack = [](const uint4& w4, float (&x)[E]) {
+    const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      x[2 * t] = __uint_as_float(w[t] << 16);
+      x[2 * t + 1] = __uint_as_float(w[t] & 0xFFFF0000u);
+    }
+  };
+
+  for (int h0 = 0; h0 < p.group; h0 += kDecodeHeads) {
+    const int nh = min(kDecodeHeads, p.group - h0);
+    float q[kDecodeHeads][E];
+#pragma unroll
+    for (int hh = 0; hh < kDecodeHeads; ++hh) {
+      const int h = kh * p.group + h0 + min(hh, nh - 1);
+      const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(p.q + (size_t(b) * p.hq + h) * D + li * E));
+      unpack(w4, q[hh]);
+#pragma unroll
+      for (int e = 0; e < E; ++e) q[hh][e] *= p.scale_log2;
+    }
+    float m[kDecodeHeads], l[kDecodeHeads], o[kDecodeHeads][E];
+#pragma unroll
+    for (int hh = 0; hh < kDecodeHeads; ++hh) {
+      m[hh] = -INFINITY;
+      l[hh] = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[hh][e] = 0.f;
+    }
+    // Rows rb + rgw and rb + rgw + kRowsPerIter per iteration; the loop bound is
+    // warp-uniform so every lane reaches every shuffle.
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    uint4 ka = z, va = z, kb = z, vb = z;
+    {
+      const int r0 = r_begin + warp * GPW + rgw, r1 = r0 + kRowsPerIter;
+      if (r0 < r_end) {
+        ka = __ldg(reinterpret_cast<const uint4*>(Kb + r0 * p.row_stride));
+        va = __ldg(reinterpret_cast<const uint4*>(Vb + r0 * p.row_stride));
+      }
+      if (r1 < r_end) {
+        kb = __ldg(reinterpret_cast<const uint4*>(Kb + r1 * p.row_stride));
+        vb = __ldg(reinterpret_cast<const uint4*>(Vb + r1 * p.row_stride));
+      }
+    }
+    for (int rb = r_begin + warp * GPW; rb < r_end; rb += kStep) {
+      const int r0 = rb + rgw, r1 = r0 + kRowsPerIter;
+      const int n0 = r0 + kStep, n1 = r1 + kStep;
+      uint4 kan = z, van = z, kbn = z, vbn = z;
+      if (n0 < r_end) {
+        kan = __ldg(reinterpret_cast<const uint4*>(Kb + n0 * p.row_stride));
+        van = __ldg(reinterpret_cast<const uint4*>(Vb + n0 * p.row_stride));
+      }
+      if (n1 < r_end) {
+        kbn = __ldg(reinterpret_cast<const uint4*>(Kb + n1 * p.row_stride));
+        vbn = __ldg(reinterpret_cast<const uint4*>(Vb + n1 * p.row_stride));
+      }
+      float k0[E], v0[E], k1[E], v1[E];
+      unpack(ka, k0);
+      unpack(va, v0);
+      unpack(kb, k1);
+      unpack(vb, v1);
+      const bool ok0 = r0 < r_end, ok1 = r1 < r_end;
+#pragma unroll
+      for (int hh = 0; hh < kDecodeHeads; ++hh) {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          s0 = fmaf(q[hh][e], k0[e], s0);
+          s1 = fmaf(q[hh][e], k1[e], s1);
+        }
+#pragma unroll
+        for (int off = 1; off < LPR; off <<= 1) {
+          s0 += __shfl_xor_sync(0xffffffffu, s0, off);
+          s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+        }
+        s0 = ok0 ? s0 : -INFINITY;
+        s1 = ok1 ? s1 : -INFINITY;
+        const float m_new = fmax3(m[hh], s0, s1);
+        if (m_new != -INFINITY) {
+          const float corr = fast_exp2(m[hh] - m_new);   // 0 on the group's first row (m = -inf)
+          const float w0 = fast_exp2(s0 - m_new);
+          const float w1 = fast_exp2(s1 - m_new);
+          l[hh] = l[hh] * corr + w0 + w1;
+#pragma unroll
+          for (int e = 0; e < E; ++e) o[hh][e] = fmaf(o[hh][e], corr, fmaf(w0, v0[e], w1 * v1[e]));
+          m[hh] = m_new;
+        }
+      }
+      ka = kan;
+      va = van;
+      kb = kbn;
+      vb = vbn;
+    }
+    // Merge the GPW row groups of the warp (lanes li + LPR * g).
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+      for (int hh = 0; hh < kDecodeHeads; ++hh) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m[hh], off);
+        const float l2 = __shfl_xor_sync(0xffffffffu, l[hh], off);
+        float o2[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) o2[e] = __shfl_xor_sync(0xffffffffu, o[hh][e], off);
+        softmax_merge<E>(m[hh], l[hh], o[hh], m2, l2, o2);
+      }
+    }
+    if (rgw == 0) {
+#pragma unroll
+      for (int hh = 0; hh < kDecodeHeads; ++hh) {
+        if (li == 0) {
+          sm_m[warp][hh] = m[hh];
+          sm_l[warp][hh] = l[hh];
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) sm_o[warp][hh][li * E + e] = o[hh][e];
+      }
+    }
+    __syncthreads();
+    // The CTA's partial state of each head, merged over the warps in warp
+    // order, to the workspace: [b, h, split] = (o[0..D), m, l).
+    for (int i = threadIdx.x; i < kDecodeHeads * D; i += kDecodeThreads) {
+      const int hh = i / D, e = i - hh * D;
+      if (hh >= nh) continue;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w2 = 0; w2 < kDecodeWarps; ++w2) M = fmaxf(M, sm_m[w2][hh]);
+      float ll = 0.f, oo = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < kDecodeWarps; ++w2) {
+        const float c = M == -INFINITY ? 0.f : fast_exp2(sm_m[w2][hh] - M);
+        ll = fmaf(sm_l[w2][hh], c, ll);
+        oo = fmaf(sm_o[w2][hh][e], c, oo);
+      }
+      const int h = kh * p.group + h0 + hh;
+      float* dst = part + ((size_t(b) * p.hq + h) * p.splits + split) * (D + 2);
+      dst[e] = oo;
+      if (e == 0) {
+        dst[D] = M;
+        dst[D + 1] = ll;
+      }
+    }
+    __syncthreads();   // the warps' states are read before the next head group overwrites them
+  }
+}
+
+// Merge of the split-K partial states: one CTA of D threads per (sequence,
+// query head), thread e combining element e of every split in split order.
+template <int D>
+__global__ void __launch_bounds__(D) decode_merge_kernel(const float* part, int hq, int splits, __nv_bfloat16* O,
+                                                         float* LSE) {
+  const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
+  const float* src = part + (size_t(b) * hq + h) * splits * (D + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, src[size_t(s) * (D + 2) + D]);
+  float ll = 0.f, oo = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float* ps = src + size_t(s) * (D + 2);
+    const float c = M == -INFINITY ? 0.f : fast_exp2(ps[D] - M);
+    ll = fmaf(ps[D + 1], c, ll);
+    oo = fmaf(ps[e], c, oo);
+  }
+  const float inv = ll > 0.f ? 1.f / ll : 0.f;
+  O[(size_t(b) * hq + h) * D + e] = __float2bfloat16_rn(oo * inv);
+  if (e == 0) LSE[size_t(b) * hq + h] = ll > 0.f ? (M + fast_log2(ll)) * 0.69314718055994531f : -INFINITY;
+}
+
 }  // namespace lt

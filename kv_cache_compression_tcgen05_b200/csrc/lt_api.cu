@@ -47,6 +47,11 @@ struct DeviceInfo {
   int sm_count = 0;
   unsigned* status = nullptr;  // device address of g_status_word
   int max_decode_splits = 8;   // largest cluster the decode kernels launch with
+  // The head_dim-128 attention kernels move registers between warpgroups with
+  // setmaxnreg, which is only safe when the compiled kernels launch with the
+  // per-thread count the split was computed from (else a raise could wait
+  // forever); checked once per device.
+  bool attn128_regs_ok = false;
 };
 
 std::mutex g_mutex;
@@ -78,6 +83,15 @@ lt_status device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(lt::lazy_ratio_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              lt::RatioLayout<128>::kBytes) != cudaSuccess)
       return LT_ERR_CUDA;
+    {
+      cudaFuncAttributes fa0{}, fa1{};
+      info.attn128_regs_ok =
+          cudaFuncGetAttributes(&fa0, lt::attn_fwd_kernel<128, false>) == cudaSuccess &&
+          cudaFuncGetAttributes(&fa1, lt::attn_fwd_kernel<128, true>) == cudaSuccess &&
+          fa0.numRegs == lt::AttnLayout<128>::kLaunchRegs && fa1.numRegs == lt::AttnLayout<128>::kLaunchRegs &&
+          2 * lt::AttnLayout<128>::kRegsSoftmax + lt::AttnLayout<128>::kRegsOther ==
+              3 * lt::AttnLayout<128>::kLaunchRegs;
+    }
     // Clusters of 16 CTAs are beyond the portable size: use them for the decode
     // split only where the device reports that one fits.
     info.max_decode_splits = 8;
@@ -220,6 +234,7 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
 
   if (!dev && (st = device_info(&dev)) != LT_OK) return st;
   const int d = shape->head_dim;
+  if (d == 128 && !dev->attn128_regs_ok) return LT_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv;
   if (make_map(&mq, Q, d, shape->hq, T) != LT_OK || make_map(&mk, K, d, shape->hkv, T) != LT_OK ||
       make_map(&mv, V, d, shape->hkv, T) != LT_OK)
@@ -695,6 +710,74 @@ lt_status lt_decode_attn(const void* q, const void* K, const void* V, const int3
   p.O = static_cast<__nv_bfloat16*>(O);
   p.LSE = LSE;
   return launch_decode(p, head_dim, max_len, softmax_scale, stream);
+}
+
+size_t lt_decode_splitk_workspace_bytes(int batch, int hq, int head_dim, int max_len) {
+  if (batch < 1 || hq < 1 || (head_dim != 64 && head_dim != 128) || max_len < 1) return 0;
+  return lt::decode_splitk_floats(batch, hq, head_dim, max_len) * sizeof(float);
+}
+
+namespace {
+
+// Checks and launches of the split-K decode over a full cache; `part` holds
+// at least lt_decode_splitk_workspace_bytes of the call's sizes.
+lt_status launch_decode_splitk(const void* q, const void* K, const void* V, const int32_t* seq_start,
+                               int seq_capacity, const int32_t* len, int batch, int hq, int hkv, int head_dim,
+                               int max_len, void* O, float* LSE, float softmax_scale, float* part,
+                               lt_stream stream) {
+  if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(len, 4) || !aligned(O, 16) ||
+      !aligned(LSE, 4) || !aligned(part, 16) || (seq_start && !aligned(seq_start, 4)) || batch < 1 ||
+      batch > 65535 || hq < 1 || hkv < 1 || hq % hkv || max_len < 1 || (!seq_start && seq_capacity < max_len) ||
+      !std::isfinite(softmax_scale))
+    return LT_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return LT_ERR_UNSUPPORTED;
+  const int splits = lt::decode_splitk_splits(max_len);
+  if ((long long)hkv * splits > 2147483647LL) return LT_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  lt_status st = device_info(&dev);
+  if (st != LT_OK) return st;
+  lt::DecodeParams p{};
+  p.batch = batch;
+  p.hq = hq;
+  p.hkv = hkv;
+  p.group = hq / hkv;
+  p.splits = splits;
+  p.max_len = max_len;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.K = static_cast<const __nv_bfloat16*>(K);
+  p.V = static_cast<const __nv_bfloat16*>(V);
+  p.seq_start = seq_start;
+  p.row_stride = (long long)hkv * head_dim;
+  p.seq_stride = seq_start ? 0 : (long long)seq_capacity * p.row_stride;
+  p.head_stride = head_dim;
+  p.len = len;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.LSE = LSE;
+  p.scale_log2 = resolve_scale(softmax_scale, head_dim) * kLog2e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid(hkv * splits, batch, 1), mgrid(hq, batch, 1);
+  if (head_dim == 64) {
+    lt::decode_splitk_kernel<64><<<grid, lt::kDecodeThreads, 0, s>>>(p, part);
+    lt::decode_merge_kernel<64><<<mgrid, 64, 0, s>>>(part, hq, splits, p.O, LSE);
+  } else {
+    lt::decode_splitk_kernel<128><<<grid, lt::kDecodeThreads, 0, s>>>(p, part);
+    lt::decode_merge_kernel<128><<<mgrid, 128, 0, s>>>(part, hq, splits, p.O, LSE);
+  }
+  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+}
+
+}  // namespace
+
+lt_status lt_decode_attn_splitk(const void* q, const void* K, const void* V, const int32_t* seq_start,
+                                int seq_capacity, const int32_t* len, int batch, int hq, int hkv, int head_dim,
+                                int max_len, void* O, float* LSE, float softmax_scale, void* workspace,
+                                size_t workspace_bytes, lt_stream stream) {
+  LT_RANGE();
+  const size_t need = lt_decode_splitk_workspace_bytes(batch, hq, head_dim, max_len);
+  if (need == 0 && (head_dim == 64 || head_dim == 128)) return LT_ERR_INVALID_ARG;
+  if (need > 0 && (!workspace || workspace_bytes < need)) return LT_ERR_INVALID_ARG;
+  return launch_decode_splitk(q, K, V, seq_start, seq_capacity, len, batch, hq, hkv, head_dim, max_len, O, LSE,
+                              softmax_scale, static_cast<float*>(workspace), stream);
 }
 
 lt_status lt_selftest_wait_timeout(unsigned limit_us, lt_stream stream) {

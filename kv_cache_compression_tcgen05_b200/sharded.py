@@ -126,14 +126,14 @@ class PrefillStep:
 
     The step owns O/LSE scratch, the per-layer ratios, the device queue and
     the streaming-KV pool [budget, batch, hkv, S+W, d] of the demoted layers
-    (this rank's heads).  Without a process group the queue push rides on the
-    attention kernel (lt_prefill_attn_ratio_push), so a layer is two library
-    launches.  The step's buffers are created on the current stream: a step
+    (this rank's heads).  A layer is three library launches (attention with
+    the ratio, queue push, compaction or slot commit), or two with
+    fused_push=True.  The step's buffers are created on the current stream: a step
     enqueued on another stream must be ordered after them and after the
     inputs (e.g. stream.wait_stream(torch.cuda.current_stream()))."""
 
     def __init__(self, layers, budget, S, W, n_obs, cu_seqlens=None, max_seqlen=None, group=None, kv_pool=False,
-                 dims=None, fused_push=True):
+                 dims=None, fused_push=False):
         if not layers:
             raise ValueError("at least one layer is required")
         if any(lay is not None and len(lay) != 3 for lay in layers):
@@ -169,9 +169,13 @@ class PrefillStep:
         self.T, self.hq, self.hkv, self.d = T, hq, hkv, d
         self.group = group
         self.kv_pool = bool(kv_pool)
-        # The queue push rides on the attention kernel (its last CTA) unless
-        # the heads are split (the push then follows the ratio exchange) or
-        # fused_push=False (a separate push launch, e.g. to compare the two).
+        # fused_push: the queue push rides on the attention kernel's last CTA
+        # (lt_prefill_attn_ratio_push; two launches per layer) instead of its
+        # own launch.  Off by default: measured on B200 the separate push,
+        # launched programmatically behind the attention, costs less than the
+        # completion count every CTA then takes (gqa1p2b step 1.88 against
+        # 1.91 ms; equal at long128k).  With the heads split the push follows
+        # the ratio exchange, so it is always separate.
         self.fused_push = bool(fused_push) and group is None
         self.world = torch.distributed.get_world_size(group) if group is not None else 1
         self.batch = cu_seqlens.numel() - 1 if cu_seqlens is not None else 1

@@ -166,7 +166,13 @@ def test_pool_step_matches_oracle_and_resident_step():
     assert torch.equal(order, order_r) and torch.equal(pool.ratio, resident.ratio)
     assert torch.equal(pool.K_pool, resident.K_pool) and torch.equal(pool.V_pool, resident.V_pool)
     assert torch.equal(pool.pool_len, resident.pool_len)
-    assert pool.kernel_launches() == 1 + 2 * cfg.layers
+    assert pool.kernel_launches() == 1 + 3 * cfg.layers
+    # The queue push fused into the attention kernel gives the same step, bit for bit.
+    fused = lt.PrefillStep(layers, cfg.budget, cfg.S, cfg.W, cfg.n_obs, kv_pool=True, fused_push=True)
+    _, order_f = _run(fused)
+    assert fused.kernel_launches() == 1 + 2 * cfg.layers
+    assert torch.equal(order, order_f) and torch.equal(pool.ratio, fused.ratio)
+    assert torch.equal(pool.K_full, fused.K_full) and torch.equal(pool.K_pool, fused.K_pool)
 
 
 def test_pool_step_packed_batch_per_sequence_slots():

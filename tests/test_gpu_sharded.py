@@ -210,7 +210,7 @@ def test_sequence_slices_match_full_batch(world):
 def test_prefill_step_with_budget_zero_demotes_nothing():
     cfg = _cfg()
     step = lt.PrefillStep(_layers(cfg), 0, cfg.S, cfg.W, cfg.n_obs)
-    assert step.kernel_launches() == 1 + cfg.layers          # attention with the push; no compaction launches
+    assert step.kernel_launches() == 1 + 2 * cfg.layers      # attention and push; no compaction launches
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     step.enqueue(s)

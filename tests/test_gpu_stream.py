@@ -229,3 +229,59 @@ def test_full_decode_rejects_bad_args():
         lt.lt_decode_attn(q, K, K, ln, max_len=17)
     with pytest.raises(ValueError):            # packed cache without seq_start
         lt.lt_decode_attn(q, K[0], K[0], ln)
+
+
+# ------------------------------------------------------------ split-K decode
+
+@pytest.mark.parametrize("B,cap,hq,hkv,d", [(6, 300, 8, 2, 64), (3, 20000, 8, 8, 128), (2, 70, 6, 3, 128),
+                                             (1, 9000, 16, 8, 64), (1, 40000, 32, 8, 128)])
+def test_splitk_decode_padded_cache_matches_oracle(B, cap, hq, hkv, d):
+    """The split-K decode (many CTAs per (sequence, KV head), partial states in
+    a workspace, merged in split order) against the oracle on ragged lengths
+    (0, 1, the whole capacity, and ones that leave splits empty)."""
+    g = torch.Generator(device="cuda").manual_seed(cap + d + 1)
+    q = torch.randn((B, hq, d), generator=g, device="cuda").bfloat16()
+    K = (torch.randn((B, cap, hkv, d), generator=g, device="cuda") * 1.2).bfloat16()
+    V = torch.randn((B, cap, hkv, d), generator=g, device="cuda").bfloat16()
+    lens = [cap, 0, 1, cap // 3, cap - 1, 129][:B]
+    ln = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    O, L = lt.lt_decode_attn_splitk(q, K, V, ln)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle_decode_full(q, K.reshape(B * cap, hkv, d), V.reshape(B * cap, hkv, d),
+                                      [b * cap for b in range(B)], lens)
+    compare(O, L, O_ref, L_ref)
+    # Deterministic: the same bits on a second call with a dirty workspace.
+    ws = torch.full((lt.lt_decode_splitk_workspace_bytes(B, hq, d, cap),), 0x7F, dtype=torch.uint8, device="cuda")
+    O2, L2 = lt.lt_decode_attn_splitk(q, K, V, ln, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(O, O2) and torch.equal(L, L2)
+
+
+def test_splitk_decode_of_last_row_equals_prefill():
+    """Packed prefill K/V of a long and a short sequence: decoding each
+    sequence's last prefill query gives the prefill's own last-row O and LSE."""
+    cfg = synth.custom(seqlens=(33000, 700), hq=8, hkv=2, d=128, S=4, W=64, n_obs=8, seed=19)
+    Q, K, V = synth.layer_inputs(cfg, 0, "cuda")
+    O_pf, LSE_pf = gpu_attention(cfg, Q, K, V)
+    cu_h = np.array(cfg.cu_seqlens(), np.int32)
+    starts = torch.tensor(cu_h[:-1], dtype=torch.int32, device="cuda")
+    ln = torch.tensor(np.diff(cu_h), dtype=torch.int32, device="cuda")
+    last = torch.tensor(cu_h[1:] - 1, device="cuda", dtype=torch.long)
+    q = Q[last].contiguous()
+    O, L = lt.lt_decode_attn_splitk(q, K, V, ln, seq_start=starts, max_len=cfg.max_seqlen)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle_decode_full(q, K, V, cu_h[:-1], np.diff(cu_h))
+    compare(O, L, O_ref, L_ref)
+    assert (L - LSE_pf[:, last].T).abs().max().item() <= 2 * LSE_ABS
+    diff = (O.float() - O_pf[last].float()).norm() / O_pf[last].float().norm()
+    assert diff.item() <= 2 * O_REL_L2
+
+
+def test_splitk_decode_rejects_a_small_workspace():
+    q = torch.zeros((1, 4, 64), dtype=torch.bfloat16, device="cuda")
+    K = torch.zeros((1, 5000, 2, 64), dtype=torch.bfloat16, device="cuda")
+    ln = torch.full((1,), 5000, dtype=torch.int32, device="cuda")
+    need = lt.lt_decode_splitk_workspace_bytes(1, 4, 64, 5000)
+    assert need == 4 * 5 * (64 + 2) * 4          # 4 heads, ceil(5000 / 1024) = 5 splits
+    with pytest.raises(lt.LtError):
+        lt.lt_decode_attn_splitk(q, K, K, ln, workspace=torch.empty(need - 16, dtype=torch.uint8, device="cuda"))
