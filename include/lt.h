@@ -408,6 +408,30 @@ lt_status lt_decode_attn_splitk(const void* q, const void* K, const void* V, con
                                 size_t workspace_bytes, lt_stream stream);
 
 /*
+ * lt_decode_attn_splitk for callers that cannot allocate device memory when
+ * they decode -- e.g. a plugin whose host framework owns all device memory,
+ * or a serving loop where cudaMalloc's implicit synchronisation is not
+ * allowed.  (The pages have no counterpart: this is an interface choice of
+ * this library.)  Same arguments, results and errors as lt_decode_attn_splitk
+ * without the workspace: the partial states go to a fixed array inside the
+ * library's own device memory, lt_decode_splitk_noalloc_capacity_bytes()
+ * bytes (4 MiB), which every device that loads the library holds until the
+ * process exits.  A call whose lt_decode_splitk_workspace_bytes(batch, hq,
+ * head_dim, max_len) exceeds it returns LT_ERR_INVALID_ARG and enqueues
+ * nothing.  Nothing is allocated: the first library call on a device (this
+ * one or any other) looks up the array's device address once, so make that
+ * first call before any stream capture.  All calls on a device share the
+ * array and it keeps the last call's contents; nothing in it needs to start
+ * at zero, but calls that overlap on the GPU (other streams, or graphs
+ * replayed concurrently) race on it and must be serialised by the caller.
+ */
+size_t lt_decode_splitk_noalloc_capacity_bytes(void);
+lt_status lt_decode_attn_splitk_noalloc(const void* q, const void* K, const void* V, const int32_t* seq_start,
+                                        int seq_capacity, const int32_t* len, int batch, int hq, int hkv,
+                                        int head_dim, int max_len, void* O, float* LSE, float softmax_scale,
+                                        lt_stream stream);
+
+/*
  * Device status word of the current device: LT_OK, or LT_ERR_TIMEOUT if a kernel
  * gave up a bounded wait since the last clear.  Synchronises the device.
  * clear != 0 resets the word.

@@ -53,6 +53,8 @@ from .binding import (  # noqa: F401
     lt_stream_decode,
     lt_decode_attn,
     lt_decode_attn_splitk,
+    lt_decode_attn_splitk_noalloc,
+    lt_decode_splitk_noalloc_capacity_bytes,
     lt_decode_splitk_workspace_bytes,
     lt_stream_ring_init,
 )

@@ -72,6 +72,8 @@ _SIGS = {
     "lt_stream_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp]),
     "lt_decode_attn": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp]),
     "lt_decode_splitk_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i]),
+    "lt_decode_splitk_noalloc_capacity_bytes": (ctypes.c_size_t, []),
+    "lt_decode_attn_splitk_noalloc": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp]),
     "lt_decode_attn_splitk": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _vp, _vp, _f, _vp,
                                    ctypes.c_size_t, _vp]),
     "lt_device_status": (_i, [_i]),
@@ -681,4 +683,29 @@ def lt_decode_attn_splitk(q, K, V, seq_len, seq_start=None, max_len=None, softma
                                            0.0 if softmax_scale is None else float(softmax_scale),
                                            workspace.data_ptr(), workspace.numel(), _stream_handle(stream)),
            "lt_decode_attn_splitk")
+    return out, lse
+
+
+def lt_decode_splitk_noalloc_capacity_bytes() -> int:
+    return int(library().lt_decode_splitk_noalloc_capacity_bytes())
+
+
+def lt_decode_attn_splitk_noalloc(q, K, V, seq_len, seq_start=None, max_len=None, softmax_scale=None, out=None,
+                                  lse=None, stream=None):
+    """lt_decode_attn_splitk with the library's fixed workspace instead of one
+    the caller allocates (see include/lt.h): for callers that cannot allocate
+    device memory at decode time.  Raises ValueError, before any launch, when
+    the call's workspace would exceed the fixed capacity."""
+    q, K, V, seq_start, cap, seq_len, B, hq, hkv, d, limit, out, lse = _decode_full_args(
+        q, K, V, seq_len, seq_start, max_len, out, lse)
+    need, have = lt_decode_splitk_workspace_bytes(B, hq, d, limit), lt_decode_splitk_noalloc_capacity_bytes()
+    if need > have:
+        raise ValueError(f"split-K decode of batch {B}, {hq} heads, head_dim {d}, {limit} rows needs {need} bytes "
+                         f"of workspace; the allocation-free entry point holds {have}")
+    _check(library().lt_decode_attn_splitk_noalloc(q.data_ptr(), K.data_ptr(), V.data_ptr(),
+                                                   None if seq_start is None else seq_start.data_ptr(), cap,
+                                                   seq_len.data_ptr(), B, hq, hkv, d, limit, out.data_ptr(),
+                                                   lse.data_ptr(), 0.0 if softmax_scale is None else
+                                                   float(softmax_scale), _stream_handle(stream)),
+           "lt_decode_attn_splitk_noalloc")
     return out, lse

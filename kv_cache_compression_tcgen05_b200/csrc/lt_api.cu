@@ -40,6 +40,13 @@ struct CallRange {
 // bounded wait.  One copy per device; read and cleared by lt_device_status.
 __device__ unsigned g_status_word;
 
+// Workspace of lt_decode_attn_splitk_noalloc: a fixed array in the library's
+// own device memory, for callers that cannot allocate.  Every device that
+// loads the library holds it until the process exits; every call on a device
+// shares it.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // 4 MiB
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
 constexpr int kMaxDevices = 64;
 
 struct DeviceInfo {
@@ -52,6 +59,9 @@ struct DeviceInfo {
   // per-thread count the split was computed from (else a raise could wait
   // forever); checked once per device.
   bool attn128_regs_ok = false;
+  // Device address of g_noalloc_scratch (host code may not use the symbol
+  // itself: on the host it names a stand-in, not device memory).
+  float* noalloc_scratch = nullptr;
 };
 
 std::mutex g_mutex;
@@ -70,6 +80,9 @@ lt_status device_info(DeviceInfo** out) {
     void* addr = nullptr;
     if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess) return LT_ERR_CUDA;
     info.status = static_cast<unsigned*>(addr);
+    void* scratch = nullptr;
+    if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || !scratch) return LT_ERR_CUDA;
+    info.noalloc_scratch = static_cast<float*>(scratch);
     if (cudaFuncSetAttribute(lt::attn_fwd64_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              lt::Attn64Layout::kAlloc) != cudaSuccess ||
         cudaFuncSetAttribute(lt::attn_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -778,6 +791,23 @@ lt_status lt_decode_attn_splitk(const void* q, const void* K, const void* V, con
   if (need > 0 && (!workspace || workspace_bytes < need)) return LT_ERR_INVALID_ARG;
   return launch_decode_splitk(q, K, V, seq_start, seq_capacity, len, batch, hq, hkv, head_dim, max_len, O, LSE,
                               softmax_scale, static_cast<float*>(workspace), stream);
+}
+
+size_t lt_decode_splitk_noalloc_capacity_bytes(void) { return kNoAllocScratchBytes; }
+
+lt_status lt_decode_attn_splitk_noalloc(const void* q, const void* K, const void* V, const int32_t* seq_start,
+                                        int seq_capacity, const int32_t* len, int batch, int hq, int hkv,
+                                        int head_dim, int max_len, void* O, float* LSE, float softmax_scale,
+                                        lt_stream stream) {
+  LT_RANGE();
+  const size_t need = lt_decode_splitk_workspace_bytes(batch, hq, head_dim, max_len);
+  if (need == 0 && (head_dim == 64 || head_dim == 128)) return LT_ERR_INVALID_ARG;
+  if (need > kNoAllocScratchBytes) return LT_ERR_INVALID_ARG;   // beyond the fixed workspace
+  DeviceInfo* dev = nullptr;
+  lt_status st = device_info(&dev);   // the first call on a device takes the array's address
+  if (st != LT_OK) return st;
+  return launch_decode_splitk(q, K, V, seq_start, seq_capacity, len, batch, hq, hkv, head_dim, max_len, O, LSE,
+                              softmax_scale, dev->noalloc_scratch, stream);
 }
 
 lt_status lt_selftest_wait_timeout(unsigned limit_us, lt_stream stream) {
