@@ -437,6 +437,7 @@ def run_ours(args, cfg, rank, world):
             lt.lt_prefill_attn(Q, K, V, out=pf.O, lse=pf.LSE, **kw)
             e1.record()
             lt.lt_lazy_ratio(Q, K, pf.LSE, cfg.S, cfg.W, cfg.n_obs, out=ratio_out, **kw)
+            e2.record()
             ratio_out.zero_()      # outside the fused launch's events (accumulate form, as in the step)
             e2b = torch.cuda.Event(enable_timing=True)
             e2b.record()

@@ -476,24 +476,28 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
         }
         // exp2 in 32-column chunks; each chunk's bf16 P goes to TMEM (16
         // columns) as soon as it is packed.
-        float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // The scale/shift and the row sum use the packed two-lane fp32
+        // instructions (one issue slot per pair of columns).
+        float2 sum4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const float2 sl2x2 = make_float2(sl2, sl2), neg_mx2 = make_float2(neg_m, neg_m);
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int c0 = cb * 32 + 2 * c;
-            const float x0 = fmaf(__uint_as_float(sr[c0]), sl2, neg_m);
-            const float x1 = fmaf(__uint_as_float(sr[c0 + 1]), sl2, neg_m);
-            const float p0 = fast_exp2(x0);
-            const float p1 = fast_exp2(x1);
-            sum8[c & 7] += p0 + p1;
+            const float2 xx = fma_f32x2(make_float2(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1])), sl2x2,
+                                        neg_mx2);
+            const float p0 = fast_exp2(xx.x);
+            const float p1 = fast_exp2(xx.y);
+            sum4[c & 3] = add_f32x2(sum4[c & 3], make_float2(p0, p1));
             pk[c] = pack_bf16x2(p0, p1);
           }
           tmem_st16(s_col + cb * 16, pk);
         }
-        const float tile_sum =
-            ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+        const float2 s01 = add_f32x2(sum4[0], sum4[1]), s23 = add_f32x2(sum4[2], sum4[3]);
+        const float2 s0123 = add_f32x2(s01, s23);
+        const float tile_sum = s0123.x + s0123.y;
         l_run += tile_sum;
         if constexpr (kRatio) {
           if (whole) num += tile_sum;
