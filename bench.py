@@ -700,6 +700,21 @@ def measure_e2e(args, cfg, lt, pf, world, job_flops, long_step):
     layer's K/V stays on the device (the KV cache the queue manages).  `cfg`
     is this rank's shape (its slice when the heads or sequences are split);
     job_flops the work of the whole job per step."""
+    # Every rank of a node pins its own copy of the inputs: check that the host
+    # has room for all of them before pinning (a failed pin would end the run).
+    need = sum(t.numel() * t.element_size() for lay in pf.layers for t in lay)
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = None
+    local = int(os.environ.get("LOCAL_WORLD_SIZE", world))
+    skip = avail is not None and need * local > 0.7 * avail
+    if max_over_ranks(1.0 if skip else 0.0, world) > 0:     # every rank takes the same branch
+        avail = avail or 0
+        return {"value": None, "unit": "TFLOP/s", "h2d_bytes_per_step": int(need), "d2h_bytes_per_step": 0,
+                "skipped": f"{local} rank(s) x {need / 2**30:.1f} GiB of pinned inputs exceed 70% of the host's "
+                           f"{avail / 2**30:.0f} GiB available"}
     host = []
     for lay in pf.layers:
         host.append(tuple(torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t) for t in lay))

@@ -62,6 +62,7 @@ struct AttnParams {
   int group;        // hq / hkv
   int n_qtiles;     // ceil(max_seqlen / 128)
   int pair_heads;   // 1: an item pairs two heads; 0: it pairs two q-tiles
+  int qt_band;      // > 0 (with pair_heads): items ordered by q-tile bands of this many tiles, KV head by KV head
   int num_items;
   const int32_t* cu_seqlens;  // device [batch+1] or null (one sequence)
   __nv_bfloat16* O;
@@ -113,6 +114,30 @@ struct AttnItem {
   bool hasB;
 };
 
+// Fused ratio's masked sum of one key tile, in fp32 from the tile's scores
+// (scores sr, scale sl2 and shift neg_m as the exponential loop uses them):
+// the weights of the sink columns c < sink_c (the same for every row of the
+// tile) and of the window columns c >= max(win_c, sink_c), for threads whose
+// `part` is set (0 for the others).  Only those columns are exponentiated:
+// columns below sink_c and from the smallest first window column of the
+// warp's rows on (both bounds warp-uniform: each column's test is a uniform
+// branch, and the unrolled loop indexes the scores with constants).  The
+// whole warp calls it.
+__device__ __forceinline__ float masked_score_sum(const uint32_t (&sr)[128], float sl2, float neg_m, int sink_c,
+                                                  int win_c, bool part) {
+  float acc = 0.f;
+  const int w0 = max(win_c, sink_c);
+  const int lo = int(__reduce_min_sync(0xffffffffu, unsigned(part ? max(w0, 0) : 128)));
+#pragma unroll
+  for (int c = 0; c < 128; ++c) {
+    if (c < sink_c || c >= lo) {   // warp-uniform: sink_c and lo are the same in every lane
+      const float w = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, neg_m));
+      acc += (c < sink_c || c >= w0) ? w : 0.f;
+    }
+  }
+  return part ? acc : 0.f;
+}
+
 __device__ __forceinline__ void seq_bounds(const AttnParams& p, int b, int& start, int& len) {
   if (p.cu_seqlens) {
     start = p.cu_seqlens[b];
@@ -127,6 +152,34 @@ __device__ __forceinline__ void seq_bounds(const AttnParams& p, int b, int& star
 // Items are ordered heaviest first; the items of one q position are consecutive
 // (heads of a sequence next to each other, so concurrent CTAs share K/V in L2).
 __device__ __forceinline__ bool attn_decode(const AttnParams& p, int t, AttnItem& it) {
+  if (p.pair_heads && p.qt_band > 0) {
+    // Long sequences: q-tiles in bands of qt_band (heaviest band first), and
+    // within a band one KV head after another, so the CTAs running at the same
+    // time stream the same KV head's K/V (which then stays in L2) instead of
+    // every KV head's at once.
+    const int ppk = p.group >> 1;                       // head pairs per KV head
+    const int per_qt = p.batch * ppk;
+    const int per_kh = p.qt_band * per_qt;
+    const int per_band = per_kh * p.hkv;
+    const int band = t / per_band;
+    int rem = t - band * per_band;
+    const int kh = rem / per_kh;
+    rem -= kh * per_kh;
+    const int qin = rem / per_qt;
+    rem -= qin * per_qt;
+    it.b = rem / ppk;
+    const int hp = kh * ppk + (rem - it.b * ppk);
+    const int qt = p.n_qtiles - 1 - (band * p.qt_band + qin);
+    if (qt < 0) return false;                           // the last band's unused places
+    seq_bounds(p, it.b, it.start, it.len);
+    it.h[0] = 2 * hp;
+    it.h[1] = 2 * hp + 1;
+    it.qt[0] = it.qt[1] = qt;
+    it.n[0] = it.n[1] = qt + 1;
+    it.hasB = true;
+    it.kh = it.h[0] / p.group;
+    return qt * 128 < it.len;
+  }
   if (p.pair_heads) {
     const int hp_count = p.hq >> 1;
     const int per_q = p.batch * hp_count;
@@ -456,22 +509,18 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
         // Keys after i carry weight 0 (causal mask), so a tile that starts
         // inside the window counts whole (its row sum, below); only the tile
         // holding the window's first key and the tile holding the sinks need
-        // a per-key mask.  That masked sum is taken before P is built, so the
-        // scores die as the exponential loop consumes them in every tile.
-        bool whole = false, part = false;
+        // a per-key mask, summed in fp32 from the scores before P is built
+        // (masked_score_sum exponentiates only the columns that count).
+        // Items with no observed row (tile_obs false, the same in every
+        // thread of the tile) skip all of it, the vote included.
+        bool whole = false;
         if constexpr (kRatio) {
-          const int win_c = qpos - p.W + 1 - j * 128;   // first window column
-          const int sink_c = p.S - j * 128;              // columns below it are sinks
-          whole = row_obs && win_c <= 0;
-          part = row_obs && !whole && (win_c < 128 || sink_c > 0);
-          if (__any_sync(0xffffffffu, part)) {
-            float acc = 0.f;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-              const float w = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, neg_m));
-              acc += (c < sink_c || c >= win_c) ? w : 0.f;
-            }
-            if (part) num += acc;
+          if (tile_obs) {
+            const int win_c = qpos - p.W + 1 - j * 128;   // first window column
+            const int sink_c = p.S - j * 128;              // columns below it are sinks
+            whole = row_obs && win_c <= 0;
+            const bool part = row_obs && !whole && (win_c < 128 || sink_c > 0);
+            if (__any_sync(0xffffffffu, part)) num += masked_score_sum(sr, sl2, neg_m, sink_c, win_c, part);
           }
         }
         // exp2 in 32-column chunks; each chunk's bf16 P goes to TMEM (16

@@ -343,18 +343,22 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
         // Fused ratio: the weights of the keys in K_i = [0, min(S, i+1)) U
         // [max(S, i-W+1), i] within this key tile (columns c = key - 128 j).
         // Keys after i carry weight 0 (causal mask), so a tile that starts
-        // inside the window counts whole (its row sum, below); only the tile
-        // holding the window's first key and the tile holding the sinks need
-        // a per-key mask, which the exponential loop applies to the weights it
-        // computes anyway (a second instance of the loop, taken warp-uniformly
-        // by those tiles only: no exponential is evaluated twice).
-        int win_c = 0, sink_c = 0;
-        bool whole = false, part = false;
+        // inside the window counts whole (added below, from the tile's row
+        // sum); only the tile holding the window's first key and the tile
+        // holding the sinks need a per-key mask, summed in fp32 from the
+        // scores before P is built (masked_score_sum exponentiates only the
+        // columns that count).  Items with no observed row (tile_obs false,
+        // the same in every thread of the tile) skip all of it, the vote
+        // included.
+        bool whole = false;
         if constexpr (kRatio) {
-          win_c = qpos - p.W + 1 - j * 128;   // first window column
-          sink_c = p.S - j * 128;              // columns below it are sinks
-          whole = row_obs && win_c <= 0;
-          part = row_obs && !whole && (win_c < 128 || sink_c > 0);
+          if (tile_obs) {
+            const int win_c = qpos - p.W + 1 - j * 128;   // first window column
+            const int sink_c = p.S - j * 128;              // columns below it are sinks
+            whole = row_obs && win_c <= 0;
+            const bool part = row_obs && !whole && (win_c < 128 || sink_c > 0);
+            if (__any_sync(0xffffffffu, part)) num += masked_score_sum(sr, sl2, neg_m, sink_c, win_c, part);
+          }
         }
         // P_x(j) in four 32-column chunks of bf16 pairs; the first two are
         // held in registers and written with the third.  Before the first
@@ -365,58 +369,40 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
         // that PV time to finish.
         float2 sum4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float2 sl2x2 = make_float2(sl2, sl2), neg_mx2 = make_float2(neg_m, neg_m);
-        auto exp_tile = [&](auto masked_tag) -> float {
-          constexpr bool kMasked = decltype(masked_tag)::value;
-          float2 msum = make_float2(0.f, 0.f);
-          uint32_t pk0[16], pk1[16];
+        uint32_t pk0[16], pk1[16];
 #pragma unroll
-          for (int cb = 0; cb < 4; ++cb) {
-            uint32_t pk[16];
+        for (int cb = 0; cb < 4; ++cb) {
+          uint32_t pk[16];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const int c0 = cb * 32 + 2 * c;
-              const float2 xx = fma_f32x2(make_float2(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1])),
-                                          sl2x2, neg_mx2);
-              // kPolyPairs of every 16 pairs go to the FMA pipe, the rest to MUFU.
-              const bool poly = (c & 15) >= 16 - kPolyPairs;
-              const float p0 = poly ? exp2_fma(xx.x) : fast_exp2(xx.x);
-              const float p1 = poly ? exp2_fma(xx.y) : fast_exp2(xx.y);
-              sum4[c & 3] = add_f32x2(sum4[c & 3], make_float2(p0, p1));
-              if constexpr (kMasked) {
-                msum.x += (c0 < sink_c || c0 >= win_c) ? p0 : 0.f;
-                msum.y += (c0 + 1 < sink_c || c0 + 1 >= win_c) ? p1 : 0.f;
-              }
-              pk[c] = pack_bf16x2(p0, p1);
-            }
-            if (cb == 2 && j > 0) {
-              ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], cnt_pv & 1, ctl));
-              ++cnt_pv;
-              tc_fence_after();
-            }
-            if (cb == 0) {
-#pragma unroll
-              for (int c = 0; c < 16; ++c) pk0[c] = pk[c];
-            } else if (cb == 1) {
-#pragma unroll
-              for (int c = 0; c < 16; ++c) pk1[c] = pk[c];
-            } else {
-              if (cb == 2) {
-                tmem_st16(p_col, pk0);
-                tmem_st16(p_col + 16, pk1);
-              }
-              tmem_st16(p_col + cb * 16, pk);
-            }
+          for (int c = 0; c < 16; ++c) {
+            const int c0 = cb * 32 + 2 * c;
+            const float2 xx = fma_f32x2(make_float2(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1])), sl2x2,
+                                        neg_mx2);
+            // kPolyPairs of every 16 pairs go to the FMA pipe, the rest to MUFU.
+            const bool poly = (c & 15) >= 16 - kPolyPairs;
+            const float p0 = poly ? exp2_fma(xx.x) : fast_exp2(xx.x);
+            const float p1 = poly ? exp2_fma(xx.y) : fast_exp2(xx.y);
+            sum4[c & 3] = add_f32x2(sum4[c & 3], make_float2(p0, p1));
+            pk[c] = pack_bf16x2(p0, p1);
           }
-          return msum.x + msum.y;
-        };
-        float part_sum = 0.f;
-        if constexpr (kRatio) {
-          if (__any_sync(0xffffffffu, part))
-            part_sum = exp_tile(std::true_type{});
-          else
-            exp_tile(std::false_type{});
-        } else {
-          exp_tile(std::false_type{});
+          if (cb == 2 && j > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], cnt_pv & 1, ctl));
+            ++cnt_pv;
+            tc_fence_after();
+          }
+          if (cb == 0) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk0[c] = pk[c];
+          } else if (cb == 1) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) pk1[c] = pk[c];
+          } else {
+            if (cb == 2) {
+              tmem_st16(p_col, pk0);
+              tmem_st16(p_col + 16, pk1);
+            }
+            tmem_st16(p_col + cb * 16, pk);
+          }
         }
         if (!ok) break;
         const float2 s01 = add_f32x2(sum4[0], sum4[1]), s23 = add_f32x2(sum4[2], sum4[3]);
@@ -425,7 +411,6 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
         l_run += tile_sum;
         if constexpr (kRatio) {
           if (whole) num += tile_sum;
-          if (part) num += part_sum;
         }
         if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll

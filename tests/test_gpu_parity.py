@@ -42,6 +42,10 @@ RAGGED = [
     dict(seqlens=(383,), hq=6, hkv=1, d=64),
     dict(seqlens=(17, 640), hq=8, hkv=8, d=128),
     dict(seqlens=(0, 5, 0, 130), hq=2, hkv=1, d=64),
+    # eight sequences with g = 8: long enough (>= 2 bands of 4 q-tiles) for the
+    # banded work order, ragged lengths
+    dict(seqlens=(1500, 1100, 1300, 1400, 1200, 1250, 1350, 1150), hq=16, hkv=2, d=64),
+    dict(seqlens=(1500, 1100, 1300, 1400, 1200, 1250, 1350, 1150), hq=16, hkv=2, d=128),
 ]
 
 
@@ -267,6 +271,7 @@ FUSED = [
     dict(seqlens=(700, 5), hq=10, hkv=2, d=64, S=0, W=1, n_obs=128),
     dict(seqlens=(500,), hq=6, hkv=2, d=128, S=16, W=1000, n_obs=37),
     dict(seqlens=(383, 260), hq=3, hkv=1, d=64, S=2, W=130, n_obs=128),
+    dict(seqlens=(1500, 1100, 1300, 1400, 1200, 1250, 1350, 1150), hq=16, hkv=2, d=128, S=4, W=200, n_obs=40),
 ]
 
 
