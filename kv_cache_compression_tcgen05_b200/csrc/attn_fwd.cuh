@@ -226,10 +226,31 @@ __device__ __forceinline__ int attn_item_index(int round, int cta, int grid) {
   return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
 }
 
+// A static assignment of work items to CTAs, computed on the host for small
+// launches (a few items per CTA, where the snake order cannot balance the
+// heaviest items, and the fused ratio's extra work on the items holding the
+// observed rows would add to the slowest CTA): CTA c runs items
+// item[off[c] .. off[c+1]) in that order.  Passed as a kernel parameter.
+constexpr int kSchedMaxItems = 1536;
+constexpr int kSchedMaxCtas = 160;
+struct AttnSchedule {
+  int used;                            // 0: the snake order over all items
+  uint16_t off[kSchedMaxCtas + 1];
+  uint16_t item[kSchedMaxItems];
+};
+
+__device__ __forceinline__ int attn_rounds(const AttnSchedule& s, const AttnParams& p, int cta, int grid) {
+  return s.used ? int(s.off[cta + 1]) - int(s.off[cta]) : (p.num_items + grid - 1) / grid;
+}
+__device__ __forceinline__ int attn_item(const AttnSchedule& s, int round, int cta, int grid) {
+  return s.used ? int(s.item[s.off[cta] + round]) : attn_item_index(round, cta, grid);
+}
+
 template <int D, bool kRatio>
 __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                    const __grid_constant__ CUtensorMap tmV, const AttnParams p,
+                    const __grid_constant__ AttnSchedule sched) {
   using Lay = AttnLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -306,8 +327,8 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
       if (lane == 0) {
         int ring = 0, nq = 0;
         bool ok = true;
-        for (int round = 0; ok && round * grid < p.num_items; ++round) {
-          const int t = attn_item_index(round, cta, grid);
+        for (int round = 0, rounds = attn_rounds(sched, p, cta, grid); ok && round < rounds; ++round) {
+          const int t = attn_item(sched, round, cta, grid);
           AttnItem it;
           if (t >= p.num_items || !attn_decode(p, t, it)) continue;
           const int qb = nq & 1;
@@ -356,8 +377,8 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
         int cnt_p0 = 0, cnt_p1 = 0;   // P tiles consumed, per tile slot
         int cnt_o0 = 0, cnt_o1 = 0;   // items finished, per tile slot
         bool ok = true;
-        for (int round = 0; ok && round * grid < p.num_items; ++round) {
-          const int t = attn_item_index(round, cta, grid);
+        for (int round = 0, rounds = attn_rounds(sched, p, cta, grid); ok && round < rounds; ++round) {
+          const int t = attn_item(sched, round, cta, grid);
           AttnItem it;
           if (t >= p.num_items || !attn_decode(p, t, it)) continue;
           const int qb = nq & 1;
@@ -438,8 +459,8 @@ __global__ void __launch_bounds__(AttnLayout<D>::kThreads, 1)
     const float sl2 = p.scale_log2;
     int cnt_s = 0, cnt_o = 0;
     bool ok = true;
-    for (int round = 0; ok && round * grid < p.num_items; ++round) {
-      const int t = attn_item_index(round, cta, grid);
+    for (int round = 0, rounds = attn_rounds(sched, p, cta, grid); ok && round < rounds; ++round) {
+      const int t = attn_item(sched, round, cta, grid);
       AttnItem it;
       if (t >= p.num_items || !attn_decode(p, t, it)) continue;
       if (x == 1 && !it.hasB) continue;

@@ -10,8 +10,11 @@
 #include <algorithm>
 #include <climits>
 #include <cmath>
+#include <cstring>
 #include <mutex>
+#include <queue>
 #include <utility>
+#include <vector>
 
 #include "attn_fwd.cuh"
 #include "attn_fwd64.cuh"
@@ -225,6 +228,132 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // Long prefills: the attention's work items in q-tile bands, KV head by KV head.
 constexpr bool kBandedOrder = true;
+// Short single-sequence prefills: the static longest-first item schedule below.
+constexpr bool kStaticSchedule = true;
+
+// Static longest-first schedule of the attention's work items (one sequence,
+// a few items per CTA).  The cost model counts quarter key-tile times: both
+// tiles of an item run side by side (one per softmax warpgroup), so a pair of
+// heads on q-tile qt costs its qt + 1 key tiles, and two q-tiles of one head
+// the mean of theirs; every item adds one tile's worth of fixed work (Q load,
+// epilogue).  With the fused ratio, the key tiles that hold a sink or the
+// first window key of an observed row take an extra masked pass over their
+// scores: half a tile at head_dim 64, where the exponentials bound the loop,
+// a quarter at 128.
+struct ScheduleKey {
+  int d, fused, n_qtiles, len, hq, pair, S, W, n_obs, grid, num_items;
+  bool operator==(const ScheduleKey& o) const {
+    return d == o.d && fused == o.fused && n_qtiles == o.n_qtiles && len == o.len && hq == o.hq &&
+           pair == o.pair && S == o.S && W == o.W && n_obs == o.n_obs && grid == o.grid &&
+           num_items == o.num_items;
+  }
+};
+
+// Key tiles of q-tile qt (rows qt*128 .. min(len, qt*128+128) - 1) whose
+// scores the fused ratio sums by a per-key mask: those below S (the sinks)
+// and, for each observed row i, the tile holding key i - W + 1 when that key
+// is not the tile's first.
+int masked_tiles(int qt, int len, int S, int W, int n_obs) {
+  const int obs_lo = len - std::min(n_obs, len);
+  const int r0 = std::max(qt * 128, obs_lo), r1 = std::min(len, qt * 128 + 128) - 1;
+  if (r0 > r1) return 0;
+  int count = std::min((S + 127) / 128, qt + 1);
+  int last = -1;
+  for (int i = r0; i <= r1; ++i) {
+    const int w = i - W + 1;
+    if (w <= 0 || (w & 127) == 0) continue;
+    const int j = w / 128;
+    if (j == last || j * 128 < S) continue;
+    count += 1;
+    last = j;
+  }
+  return count;
+}
+
+int64_t item_cost(const ScheduleKey& k, int t) {
+  const int mw = k.fused ? (k.d == 64 ? 2 : 1) : 0;
+  if (k.pair) {
+    const int qt = k.n_qtiles - 1 - t / (k.hq / 2);
+    if (qt * 128 >= k.len) return 0;
+    return 4LL * (qt + 1) + 4 + (mw ? mw * masked_tiles(qt, k.len, k.S, k.W, k.n_obs) : 0);
+  }
+  const int npairs = (k.n_qtiles + 1) / 2;
+  const int qp = npairs - 1 - t / k.hq;
+  const int t1 = 2 * qp + 1, t0 = 2 * qp;
+  if (t0 * 128 >= k.len) return 0;
+  int64_t c = 4 + (t1 * 128 < k.len ? 2LL * (t1 + 1 + t0 + 1) : 4LL * (t0 + 1));
+  if (mw) {
+    c += mw * masked_tiles(t0, k.len, k.S, k.W, k.n_obs);
+    if (t1 * 128 < k.len) c += mw * masked_tiles(t1, k.len, k.S, k.W, k.n_obs);
+  }
+  return c;
+}
+
+// Fills `out` with the longest-first assignment when its slowest CTA is
+// cheaper than the snake order's; otherwise out.used = 0.
+void build_schedule(const ScheduleKey& k, lt::AttnSchedule& out) {
+  out.used = 0;
+  const int n = k.num_items, G = k.grid;
+  std::vector<int64_t> cost(n);
+  for (int t = 0; t < n; ++t) cost[t] = item_cost(k, t);
+  int64_t snake_max = 0;
+  for (int c = 0; c < G; ++c) {
+    int64_t load = 0;
+    for (int r = 0; r * G < n; ++r) {
+      const int t = r * G + ((r & 1) ? (G - 1 - c) : c);
+      if (t < n) load += cost[t];
+    }
+    snake_max = std::max(snake_max, load);
+  }
+  std::vector<int> order(n);
+  for (int t = 0; t < n; ++t) order[t] = t;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+  // Least-loaded CTA first, the lower index on ties.
+  using Slot = std::pair<int64_t, int>;
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+  for (int c = 0; c < G; ++c) heap.push({0, c});
+  std::vector<std::vector<int>> per(G);
+  int64_t lpt_max = 0;
+  for (int t : order) {
+    Slot sl = heap.top();
+    heap.pop();
+    per[sl.second].push_back(t);
+    sl.first += cost[t];
+    lpt_max = std::max(lpt_max, sl.first);
+    heap.push(sl);
+  }
+  if (lpt_max >= snake_max) return;
+  int pos = 0;
+  for (int c = 0; c < G; ++c) {
+    out.off[c] = uint16_t(pos);
+    for (int t : per[c]) out.item[pos++] = uint16_t(t);
+  }
+  out.off[G] = uint16_t(pos);
+  out.used = 1;
+}
+
+// The schedule for a launch: the snake order (used = 0) unless the launch is
+// one sequence of known length with at most kSchedMaxItems items; the last
+// shape's schedule is kept per host thread.
+const lt::AttnSchedule& attn_schedule(const ScheduleKey& k, bool eligible) {
+  static thread_local lt::AttnSchedule none = [] {
+    lt::AttnSchedule z;
+    std::memset(&z, 0, sizeof(z));
+    return z;
+  }();
+  if (!eligible || k.num_items <= k.grid || k.num_items > lt::kSchedMaxItems || k.grid > lt::kSchedMaxCtas)
+    return none;
+  static thread_local ScheduleKey last{};
+  static thread_local bool have = false;
+  static thread_local lt::AttnSchedule sched;
+  if (!have || !(last == k)) {
+    std::memset(&sched, 0, sizeof(sched));
+    build_schedule(k, sched);
+    last = k;
+    have = true;
+  }
+  return sched;
+}
 
 }  // namespace
 
@@ -319,19 +448,25 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
   p.dq_L = dq_L;
   p.dq_layer = dq_layer;
   const int grid = int(num_items < dev->sm_count ? num_items : dev->sm_count);
+  // A single sequence whose length the host knows (no cu_seqlens) and whose
+  // items are not banded may take the static schedule.
+  const ScheduleKey key{d, ratio ? 1 : 0, int(n_qtiles), T, shape->hq, pair_heads ? 1 : 0, S, W, n_obs, grid,
+                        int(num_items)};
+  const lt::AttnSchedule& sched =
+      attn_schedule(key, kStaticSchedule && shape->batch == 1 && !shape->cu_seqlens && qt_band == 0);
   cudaError_t e;
   if (d == 64) {
     constexpr int kThreads = lt::Attn64Layout::kThreads, kSmem = lt::Attn64Layout::kAlloc;
     if (ratio)
-      e = launch_pdl(lt::attn_fwd64_kernel<true>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p);
+      e = launch_pdl(lt::attn_fwd64_kernel<true>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p, sched);
     else
-      e = launch_pdl(lt::attn_fwd64_kernel<false>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p);
+      e = launch_pdl(lt::attn_fwd64_kernel<false>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p, sched);
   } else {
     constexpr int kThreads = lt::AttnLayout<128>::kThreads, kSmem = lt::AttnLayout<128>::kAlloc;
     if (ratio)
-      e = launch_pdl(lt::attn_fwd_kernel<128, true>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p);
+      e = launch_pdl(lt::attn_fwd_kernel<128, true>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p, sched);
     else
-      e = launch_pdl(lt::attn_fwd_kernel<128, false>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p);
+      e = launch_pdl(lt::attn_fwd_kernel<128, false>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p, sched);
   }
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
 }

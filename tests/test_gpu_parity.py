@@ -272,6 +272,10 @@ FUSED = [
     dict(seqlens=(500,), hq=6, hkv=2, d=128, S=16, W=1000, n_obs=37),
     dict(seqlens=(383, 260), hq=3, hkv=1, d=64, S=2, W=130, n_obs=128),
     dict(seqlens=(1500, 1100, 1300, 1400, 1200, 1250, 1350, 1150), hq=16, hkv=2, d=128, S=4, W=200, n_obs=40),
+    # One sequence with more work items than SMs: the static longest-first
+    # schedule, over q-tile pairs of one head (odd group) and over head pairs.
+    dict(seqlens=(8000,), hq=12, hkv=4, d=64, S=4, W=700, n_obs=100),
+    dict(seqlens=(5000,), hq=16, hkv=4, d=128, S=4, W=1500, n_obs=128),
 ]
 
 
