@@ -292,207 +292,217 @@ __global__ void __launch_bounds__(Attn64Layout::kThreads, 1)
         tile_obs = qt * 128 + 127 >= obs_lo && qt * 128 < it.len;
         row_obs = tile_obs && qpos >= obs_lo && qpos < it.len;
       }
-      float m_run = -INFINITY;   // running max of scale*log2(e)*s, possibly stale by < 8
-      float l_run = 0.f;         // running sum of exp2(.. - m_run)
-      float num = 0.f;           // fused ratio numerator, same frame as l_run
-      for (int j = 0; j < n; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x], cnt_s & 1, ctl));
-        if (!ok) break;
-        ++cnt_s;
-        tc_fence_after();
-        const bool diag = j == qt;
-        uint32_t sr[128];
-        {
-          uint32_t(&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-          uint32_t(&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-          uint32_t(&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
-          uint32_t(&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
-          tmem_ld32(s_col + 0, c0);
-          tmem_ld32(s_col + 32, c1);
-          tmem_ld32(s_col + 64, c2);
-          tmem_ld32(s_col + 96, c3);
-          tmem_wait_ld();
-        }
-        if (diag) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (c > row) sr[c] = __float_as_uint(-INFINITY);
-        }
-        // Row maximum: 8 independent chains of three-input max.
-        float mx8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[8 + k]));
-#pragma unroll
-        for (int c = 16; c < 128; c += 16)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
-        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-        const float m_new = fmaxf(m_run, mx * sl2);
-        const bool need = m_new > m_run + 8.f;
-        float alpha = 1.f;
-        if (need) {
-          alpha = fast_exp2(m_run - m_new);
-          m_run = m_new;
-        }
-        l_run *= alpha;
-        if constexpr (kRatio) num *= alpha;
-        // S_x(j) is in registers: its columns may take S_x(j+1).
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[x]);
-        const float neg_m = -m_run;
-        // Fused ratio: the weights of the keys in K_i = [0, min(S, i+1)) U
-        // [max(S, i-W+1), i] within this key tile (columns c = key - 128 j).
-        // Keys after i carry weight 0 (causal mask), so a tile that starts
-        // inside the window counts whole (added below, from the tile's row
-        // sum); only the tile holding the window's first key and the tile
-        // holding the sinks need a per-key mask, summed in fp32 from the
-        // scores before P is built.  Items with no observed row (tile_obs false,
-        // the same in every thread of the tile) skip all of it, the vote
-        // included.
-        bool whole = false;
-        if constexpr (kRatio) {
-          if (tile_obs) {
-            const int win_c = qpos - p.W + 1 - j * 128;   // first window column
-            const int sink_c = p.S - j * 128;              // columns below it are sinks
-            whole = row_obs && win_c <= 0;
-            const bool part = row_obs && !whole && (win_c < 128 || sink_c > 0);
-            if (__any_sync(0xffffffffu, part)) {
-              // All 128 columns, masked by value: at head_dim 64 this measured
-              // faster than masked_score_sum's column-skipping branches.
-              float acc = 0.f;
-#pragma unroll
-              for (int c = 0; c < 128; ++c) {
-                const float w = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, neg_m));
-                acc += (c < sink_c || c >= win_c) ? w : 0.f;
-              }
-              if (part) num += acc;
-            }
-          }
-        }
-        // P_x(j) in four 32-column chunks of bf16 pairs; the first two are
-        // held in registers and written with the third.  Before the first
-        // write, P_x(j-1) V_{j-1} must be done with the P columns (and with O,
-        // before a rescale): within an item that is one phase of pv_done per
-        // key tile; the first tile follows the previous item's epilogue,
-        // which consumed the last PV's phase.  Waiting two chunks in gives
-        // that PV time to finish.
-        float2 sum4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        const float2 sl2x2 = make_float2(sl2, sl2), neg_mx2 = make_float2(neg_m, neg_m);
-        uint32_t pk0[16], pk1[16];
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int c0 = cb * 32 + 2 * c;
-            const float2 xx = fma_f32x2(make_float2(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1])), sl2x2,
-                                        neg_mx2);
-            // kPolyPairs of every 16 pairs go to the FMA pipe, the rest to MUFU.
-            const bool poly = (c & 15) >= 16 - kPolyPairs;
-            const float p0 = poly ? exp2_fma(xx.x) : fast_exp2(xx.x);
-            const float p1 = poly ? exp2_fma(xx.y) : fast_exp2(xx.y);
-            sum4[c & 3] = add_f32x2(sum4[c & 3], make_float2(p0, p1));
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-          if (cb == 2 && j > 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], cnt_pv & 1, ctl));
-            ++cnt_pv;
-            tc_fence_after();
-          }
-          if (cb == 0) {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) pk0[c] = pk[c];
-          } else if (cb == 1) {
-#pragma unroll
-            for (int c = 0; c < 16; ++c) pk1[c] = pk[c];
-          } else {
-            if (cb == 2) {
-              tmem_st16(p_col, pk0);
-              tmem_st16(p_col + 16, pk1);
-            }
-            tmem_st16(p_col + cb * 16, pk);
-          }
-        }
-        if (!ok) break;
-        const float2 s01 = add_f32x2(sum4[0], sum4[1]), s23 = add_f32x2(sum4[2], sum4[3]);
-        const float2 s0123 = add_f32x2(s01, s23);
-        const float tile_sum = s0123.x + s0123.y;
-        l_run += tile_sum;
-        if constexpr (kRatio) {
-          if (whole) num += tile_sum;
-        }
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
-          for (int cb = 0; cb < D / 32; ++cb) {
-            uint32_t o[32];
-            tmem_ld32(o_col + cb * 32, o);
+      // The tile loop and epilogue in two copies: items holding observed rows
+      // run the one with the ratio steps, all others the plain kernel's code.
+      const auto run_item = [&](auto obs) {
+        constexpr bool kObs = decltype(obs)::value;
+        float m_run = -INFINITY;   // running max of scale*log2(e)*s, possibly stale by < 8
+        float l_run = 0.f;         // running sum of exp2(.. - m_run)
+        float num = 0.f;           // fused ratio numerator, same frame as l_run
+        for (int j = 0; j < n; ++j) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&s_full[x], cnt_s & 1, ctl));
+          if (!ok) break;
+          ++cnt_s;
+          tc_fence_after();
+          const bool diag = j == qt;
+          uint32_t sr[128];
+          {
+            uint32_t(&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+            uint32_t(&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+            uint32_t(&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
+            uint32_t(&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
+            tmem_ld32(s_col + 0, c0);
+            tmem_ld32(s_col + 32, c1);
+            tmem_ld32(s_col + 64, c2);
+            tmem_ld32(s_col + 96, c3);
             tmem_wait_ld();
+          }
+          if (diag) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(o_col + cb * 32, o);
+            for (int c = 0; c < 128; ++c)
+              if (c > row) sr[c] = __float_as_uint(-INFINITY);
+          }
+          // Row maximum: 8 independent chains of three-input max.
+          float mx8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[8 + k]));
+#pragma unroll
+          for (int c = 16; c < 128; c += 16)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
+          const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+          const float m_new = fmaxf(m_run, mx * sl2);
+          const bool need = m_new > m_run + 8.f;
+          float alpha = 1.f;
+          if (need) {
+            alpha = fast_exp2(m_run - m_new);
+            m_run = m_new;
+          }
+          l_run *= alpha;
+          if constexpr (kObs) num *= alpha;
+          // S_x(j) is in registers: its columns may take S_x(j+1).
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_free[x]);
+          const float neg_m = -m_run;
+          // Fused ratio: the weights of the keys in K_i = [0, min(S, i+1)) U
+          // [max(S, i-W+1), i] within this key tile (columns c = key - 128 j).
+          // Keys after i carry weight 0 (causal mask), so a tile that starts
+          // inside the window counts whole (added below, from the tile's row
+          // sum); only the tile holding the window's first key and the tile
+          // holding the sinks need a per-key mask, summed in fp32 from the
+          // scores before P is built.  Items with no observed row (tile_obs false,
+          // the same in every thread of the tile) skip all of it, the vote
+          // included.
+          bool whole = false;
+          if constexpr (kObs) {
+            {
+              const int win_c = qpos - p.W + 1 - j * 128;   // first window column
+              const int sink_c = p.S - j * 128;              // columns below it are sinks
+              whole = row_obs && win_c <= 0;
+              const bool part = row_obs && !whole && (win_c < 128 || sink_c > 0);
+              if (__any_sync(0xffffffffu, part)) {
+                // All 128 columns, masked by value: at head_dim 64 this measured
+                // faster than masked_score_sum's column-skipping branches.
+                float acc = 0.f;
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                  const float w = fast_exp2(fmaf(__uint_as_float(sr[c]), sl2, neg_m));
+                  acc += (c < sink_c || c >= win_c) ? w : 0.f;
+                }
+                if (part) num += acc;
+              }
+            }
+          }
+          // P_x(j) in four 32-column chunks of bf16 pairs; the first two are
+          // held in registers and written with the third.  Before the first
+          // write, P_x(j-1) V_{j-1} must be done with the P columns (and with O,
+          // before a rescale): within an item that is one phase of pv_done per
+          // key tile; the first tile follows the previous item's epilogue,
+          // which consumed the last PV's phase.  Waiting two chunks in gives
+          // that PV time to finish.
+          float2 sum4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          const float2 sl2x2 = make_float2(sl2, sl2), neg_mx2 = make_float2(neg_m, neg_m);
+          uint32_t pk0[16], pk1[16];
+#pragma unroll
+          for (int cb = 0; cb < 4; ++cb) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int c0 = cb * 32 + 2 * c;
+              const float2 xx = fma_f32x2(make_float2(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1])), sl2x2,
+                                          neg_mx2);
+              // kPolyPairs of every 16 pairs go to the FMA pipe, the rest to MUFU.
+              const bool poly = (c & 15) >= 16 - kPolyPairs;
+              const float p0 = poly ? exp2_fma(xx.x) : fast_exp2(xx.x);
+              const float p1 = poly ? exp2_fma(xx.y) : fast_exp2(xx.y);
+              sum4[c & 3] = add_f32x2(sum4[c & 3], make_float2(p0, p1));
+              pk[c] = pack_bf16x2(p0, p1);
+            }
+            if (cb == 2 && j > 0) {
+              ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], cnt_pv & 1, ctl));
+              ++cnt_pv;
+              tc_fence_after();
+            }
+            if (cb == 0) {
+#pragma unroll
+              for (int c = 0; c < 16; ++c) pk0[c] = pk[c];
+            } else if (cb == 1) {
+#pragma unroll
+              for (int c = 0; c < 16; ++c) pk1[c] = pk[c];
+            } else {
+              if (cb == 2) {
+                tmem_st16(p_col, pk0);
+                tmem_st16(p_col + 16, pk1);
+              }
+              tmem_st16(p_col + cb * 16, pk);
+            }
+          }
+          if (!ok) break;
+          const float2 s01 = add_f32x2(sum4[0], sum4[1]), s23 = add_f32x2(sum4[2], sum4[3]);
+          const float2 s0123 = add_f32x2(s01, s23);
+          const float tile_sum = s0123.x + s0123.y;
+          l_run += tile_sum;
+          if constexpr (kObs) {
+            if (whole) num += tile_sum;
+          }
+          if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+            for (int cb = 0; cb < D / 32; ++cb) {
+              uint32_t o[32];
+              tmem_ld32(o_col + cb * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+              tmem_st32(o_col + cb * 32, o);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[x]);
+        }
+        if (!ok) return;
+        // --------------------------------------------------------- epilogue
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_full[x], cnt_o & 1, ctl));
+        if (!ok) return;
+        ++cnt_o;
+        // The last PV's pv_done phase (complete by now): consumed so that every
+        // wait on the barrier follows the completion of the phase before it.
+        ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], cnt_pv & 1, ctl));
+        if (!ok) return;
+        ++cnt_pv;
+        tc_fence_after();
+        const bool valid = qpos < it.len;
+        const float inv_l = 1.f / l_run;
+        const size_t orow = (size_t(it.start) + qpos) * p.hq + h;
+#pragma unroll
+        for (int cb = 0; cb < D / 32; ++cb) {
+          uint32_t o[32];
+          tmem_ld32(o_col + cb * 32, o);
+          tmem_wait_ld();
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D + cb * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
           }
         }
-        tmem_wait_st();
+        if (valid)
+          p.LSE[size_t(h) * p.total_tokens + it.start + qpos] = (m_run + fast_log2(l_run)) * 0.69314718055994531f;
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[x]);
-      }
-      if (!ok) break;
-      // --------------------------------------------------------- epilogue
-      ok = __all_sync(0xffffffffu, mbar_wait(&o_full[x], cnt_o & 1, ctl));
-      if (!ok) break;
-      ++cnt_o;
-      // The last PV's pv_done phase (complete by now): consumed so that every
-      // wait on the barrier follows the completion of the phase before it.
-      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[x], cnt_pv & 1, ctl));
-      if (!ok) break;
-      ++cnt_pv;
-      tc_fence_after();
-      const bool valid = qpos < it.len;
-      const float inv_l = 1.f / l_run;
-      const size_t orow = (size_t(it.start) + qpos) * p.hq + h;
+        if (lane == 0) mbar_arrive(&o_empty[x]);
+        if constexpr (kObs) {
+          {
+            // This tile's share of mean_i r_i: its rows added in a fixed order.
+            float r = row_obs ? num * inv_l : 0.f;
 #pragma unroll
-      for (int cb = 0; cb < D / 32; ++cb) {
-        uint32_t o[32];
-        tmem_ld32(o_col + cb * 32, o);
-        tmem_wait_ld();
-        uint32_t w[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(p.O + orow * D + cb * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-        }
-      }
-      if (valid)
-        p.LSE[size_t(h) * p.total_tokens + it.start + qpos] = (m_run + fast_log2(l_run)) * 0.69314718055994531f;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[x]);
-      if constexpr (kRatio) {
-        if (tile_obs) {
-          // This tile's share of mean_i r_i: its rows added in a fixed order.
-          float r = row_obs ? num * inv_l : 0.f;
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
-          // No barrier (a sibling warp may have left on a timed-out wait): the
-          // fourth warp to finish adds the four partials in warp order.
-          if (lane == 0) {
-            ratio_part[x * 4 + wq] = r;
-            __threadfence_block();
-            if (atomicAdd(&ratio_cnt[x], 1) == 3) {
+            for (int off = 16; off > 0; off >>= 1) r += __shfl_xor_sync(0xffffffffu, r, off);
+            // No barrier (a sibling warp may have left on a timed-out wait): the
+            // fourth warp to finish adds the four partials in warp order.
+            if (lane == 0) {
+              ratio_part[x * 4 + wq] = r;
               __threadfence_block();
-              const volatile float* part = ratio_part + x * 4;
-              const float tot = (part[0] + part[1]) + (part[2] + part[3]);
-              atomicAdd(p.ratio + size_t(it.b) * p.hq + h, tot / float(n_obs_seq));
-              ratio_cnt[x] = 0;
+              if (atomicAdd(&ratio_cnt[x], 1) == 3) {
+                __threadfence_block();
+                const volatile float* part = ratio_part + x * 4;
+                const float tot = (part[0] + part[1]) + (part[2] + part[3]);
+                atomicAdd(p.ratio + size_t(it.b) * p.hq + h, tot / float(n_obs_seq));
+                ratio_cnt[x] = 0;
+              }
             }
           }
         }
-      }
+      };
+      if (tile_obs)
+        run_item(BoolTag<true>{});
+      else
+        run_item(BoolTag<false>{});
+      if (!ok) break;
     }
   }
 

@@ -236,10 +236,13 @@ constexpr bool kStaticSchedule = true;
 // tiles of an item run side by side (one per softmax warpgroup), so a pair of
 // heads on q-tile qt costs its qt + 1 key tiles, and two q-tiles of one head
 // the mean of theirs; every item adds one tile's worth of fixed work (Q load,
-// epilogue).  With the fused ratio, the key tiles that hold a sink or the
-// first window key of an observed row take an extra masked pass over their
-// scores: half a tile at head_dim 64, where the exponentials bound the loop,
-// a quarter at 128.
+// epilogue).  With the fused ratio, each key tile that holds a sink or the
+// first window key of an observed row counts two tiles more: its masked pass
+// over the scores plus the ratio steps of the other tiles of that item.  The
+// weight was measured (fused launch per layer, one process, alternating
+// builds): 1/2, 1, 2 and 4 extra tiles gave 111.1, 111.0, 109.2 and 111.1 us
+// on a gqa1p2b layer (head_dim 64); 1/4, 1/2, 1 and 2 gave 148.0, 146.1, 144.1
+// and 142.5 us on a 4096-token head_dim-128 layer.
 struct ScheduleKey {
   int d, fused, n_qtiles, len, hq, pair, S, W, n_obs, grid, num_items;
   bool operator==(const ScheduleKey& o) const {
@@ -271,7 +274,7 @@ int masked_tiles(int qt, int len, int S, int W, int n_obs) {
 }
 
 int64_t item_cost(const ScheduleKey& k, int t) {
-  const int mw = k.fused ? (k.d == 64 ? 2 : 1) : 0;
+  const int mw = k.fused ? 8 : 0;
   if (k.pair) {
     const int qt = k.n_qtiles - 1 - t / (k.hq / 2);
     if (qt * 128 >= k.len) return 0;
