@@ -107,6 +107,30 @@ lt_status lt_prefill_attn(const lt_shape* shape, const void* Q, const void* K, c
                           float* LSE, float softmax_scale, lt_stream stream);
 
 /*
+ * The assignment of attention work items to CTAs that lt_prefill_attn (fused
+ * = 0) or lt_prefill_attn_ratio (fused = 1) computes on the host for one
+ * sequence of `len` tokens passed without cu_seqlens, on a device with `grid`
+ * SMs.  Host-only and synchronous; needs no device.  The pages have no
+ * counterpart: the kernels' items are tiles of the causal attention (two query
+ * tiles of 128 rows on one K/V stream, numbered heaviest first), and this call
+ * exposes the launch's choice so that it can be checked.  A long sequence takes
+ * the banded item order and a short one, when a longest-first assignment
+ * (cost = key tiles per item, plus, with fused, the lazy ratio's masked key
+ * tiles for S, W and n_obs as in lt_prefill_attn_ratio) lowers the slowest
+ * CTA's load below the plain round-robin order's, that assignment.
+ * Writes *num_items (the launch's item count) and *used: 1 when the static
+ * assignment is used, 0 otherwise.  With *used = 1, CTA c (c < min(grid,
+ * num_items)) runs item[off[c]] .. item[off[c+1] - 1] in that order; off: host
+ * int32 [grid + 1], item: host int32 [capacity], capacity >= *num_items
+ * (LT_ERR_INVALID_ARG otherwise, after *num_items and *used are written; off
+ * and item are untouched when *used = 0).  head_dim 64 or 128, len >= 1,
+ * hq a multiple of hkv, grid >= 1; with fused, S, W and n_obs as for
+ * lt_prefill_attn_ratio.
+ */
+lt_status lt_attn_schedule(int head_dim, int fused, int len, int hq, int hkv, int S, int W, int n_obs, int grid,
+                           int* used, int* num_items, int32_t* off, int32_t* item, int capacity);
+
+/*
  * The same attention fused with the lazy ratio: O and LSE as lt_prefill_attn,
  * and ratio[b, h] as lt_lazy_ratio computes it (same S, W, n_obs and limits),
  * accumulated inside the attention's online softmax: for the observed rows the

@@ -22,6 +22,7 @@ from .binding import (  # noqa: F401
     library,
     library_path,
     lt_compact_kv,
+    lt_attn_schedule,
     lt_device_status,
     lt_layer_score,
     lt_lazy_ratio,

@@ -52,6 +52,7 @@ _SIGS = {
     "lt_lazy_ratio": (_i, [_shp, _vp, _vp, _vp, _f, _i, _i, _i, _vp, _vp]),
     "lt_layer_score": (_f, [_vp, _i]),
     "lt_select_layers": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
+    "lt_attn_schedule": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _i]),
     "lt_queue_create": (_i, [_i, _i, ctypes.POINTER(_vp)]),
     "lt_queue_push": (_i, [_vp, _i, _f, ctypes.POINTER(_i)]),
     "lt_queue_size": (_i, [_vp]),
@@ -334,6 +335,27 @@ def lt_select_layers(ratios, budget):
     _check(library().lt_select_layers(r.ctypes.data, L, B, H, int(budget), lazy.ctypes.data, order.ctypes.data),
            "lt_select_layers")
     return lazy, order[:, : int(budget)]
+
+
+def lt_attn_schedule(head_dim, len, hq, hkv, grid, S=0, W=0, n_obs=0, fused=False):
+    """The attention launch's work assignment for one sequence of `len` tokens
+    on `grid` SMs (host-only).  Returns (num_items, None) when the launch keeps
+    its round-robin or banded order, else (num_items, [items of CTA 0, items of
+    CTA 1, ...]) with the item indices of each CTA in run order."""
+    used, n = ctypes.c_int(0), ctypes.c_int(0)
+    st = library().lt_attn_schedule(int(head_dim), 1 if fused else 0, int(len), int(hq), int(hkv), int(S), int(W),
+                                    int(n_obs), int(grid), ctypes.byref(used), ctypes.byref(n), None, None, 0)
+    if st == LT_ERR_INVALID_ARG and used.value == 1:
+        off = np.empty(int(grid) + 1, np.int32)
+        item = np.empty(max(n.value, 1), np.int32)
+        st = library().lt_attn_schedule(int(head_dim), 1 if fused else 0, int(len), int(hq), int(hkv), int(S),
+                                        int(W), int(n_obs), int(grid), ctypes.byref(used), ctypes.byref(n),
+                                        off.ctypes.data, item.ctypes.data, item.size)
+        _check(st, "lt_attn_schedule")
+        g = min(int(grid), n.value)
+        return n.value, [item[off[c]:off[c + 1]].tolist() for c in range(g)]
+    _check(st, "lt_attn_schedule")
+    return n.value, None
 
 
 def lt_queue_create(L, budget):

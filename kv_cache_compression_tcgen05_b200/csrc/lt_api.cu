@@ -338,6 +338,34 @@ void build_schedule(const ScheduleKey& k, lt::AttnSchedule& out) {
 // The schedule for a launch: the snake order (used = 0) unless the launch is
 // one sequence of known length with at most kSchedMaxItems items; the last
 // shape's schedule is kept per host thread.
+// The attention launch's work items: q-tile bands for a long single sequence
+// (see attn_decode) and the item count.  Band order for a single sequence with
+// at least two bands of q-tiles, a band being about one wave of the grid on one
+// KV head.  Shorter prefills keep the plain heaviest-first order, which
+// balances their tail, and so do packed batches: sequences of different
+// lengths leave the bands' waves partly empty (measured 5.6% slower on the
+// batched workload, against 6.9% faster on a single 131 072-token sequence).
+struct AttnPlan {
+  bool pair_heads;
+  long long n_qtiles, qt_band, num_items;
+};
+AttnPlan attn_plan(int batch, int hq, int hkv, int max_len, int sm_count) {
+  AttnPlan pl;
+  const int group = hq / hkv;
+  pl.n_qtiles = (max_len + 127) / 128;
+  pl.pair_heads = (group % 2) == 0;
+  pl.qt_band = 0;
+  if (pl.pair_heads && kBandedOrder && batch == 1) {
+    const long long band = std::max<long long>(1, sm_count / ((long long)batch * (group / 2)));
+    if (pl.n_qtiles >= 2 * band) pl.qt_band = band;
+  }
+  if (pl.qt_band > 0)
+    pl.num_items = ((pl.n_qtiles + pl.qt_band - 1) / pl.qt_band) * pl.qt_band * hkv * batch * (group / 2);
+  else
+    pl.num_items = pl.pair_heads ? pl.n_qtiles * batch * (hq / 2) : ((pl.n_qtiles + 1) / 2) * batch * hq;
+  return pl;
+}
+
 const lt::AttnSchedule& attn_schedule(const ScheduleKey& k, bool eligible) {
   static thread_local lt::AttnSchedule none = [] {
     lt::AttnSchedule z;
@@ -400,25 +428,10 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
     return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
   }
   const int group = shape->hq / shape->hkv;
-  const long long n_qtiles = (max_len + 127) / 128;
-  const bool pair_heads = (group % 2) == 0;
   if (!dev && (st = device_info(&dev)) != LT_OK) return st;
-  // Band order (see attn_decode) for a single sequence with at least two
-  // bands of q-tiles, a band being about one wave of the grid on one KV head.
-  // Shorter prefills keep the plain heaviest-first order, which balances
-  // their tail, and so do packed batches: sequences of different lengths
-  // leave the bands' waves partly empty (measured 5.6% slower on the batched
-  // workload, against 6.9% faster on a single 131 072-token sequence).
-  long long qt_band = 0;
-  if (pair_heads && kBandedOrder && shape->batch == 1) {
-    const long long band = std::max<long long>(1, dev->sm_count / ((long long)shape->batch * (group / 2)));
-    if (n_qtiles >= 2 * band) qt_band = band;
-  }
-  long long num_items;
-  if (qt_band > 0)
-    num_items = ((n_qtiles + qt_band - 1) / qt_band) * qt_band * shape->hkv * shape->batch * (group / 2);
-  else
-    num_items = pair_heads ? n_qtiles * shape->batch * (shape->hq / 2) : ((n_qtiles + 1) / 2) * shape->batch * shape->hq;
+  const AttnPlan plan = attn_plan(shape->batch, shape->hq, shape->hkv, max_len, dev->sm_count);
+  const long long n_qtiles = plan.n_qtiles, qt_band = plan.qt_band, num_items = plan.num_items;
+  const bool pair_heads = plan.pair_heads;
   if (num_items > INT_MAX) return LT_ERR_INVALID_ARG;
 
   const int d = shape->head_dim;
@@ -472,6 +485,29 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
       e = launch_pdl(lt::attn_fwd_kernel<128, false>, dim3(grid), dim3(kThreads), kSmem, s, mq, mk, mv, p, sched);
   }
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
+}
+
+lt_status lt_attn_schedule(int head_dim, int fused, int len, int hq, int hkv, int S, int W, int n_obs, int grid,
+                           int* used, int* num_items, int32_t* off, int32_t* item, int capacity) {
+  LT_RANGE();
+  if (!used || !num_items || (head_dim != 64 && head_dim != 128) || len < 1 || hq < 1 || hkv < 1 ||
+      hq % hkv != 0 || grid < 1 || capacity < 0)
+    return LT_ERR_INVALID_ARG;
+  if (fused && (S < 0 || W < 0 || (long long)S + W < 1 || n_obs < 1 || n_obs > 4096)) return LT_ERR_INVALID_ARG;
+  const AttnPlan plan = attn_plan(1, hq, hkv, len, grid);
+  if (plan.num_items > INT_MAX) return LT_ERR_INVALID_ARG;
+  *num_items = int(plan.num_items);
+  *used = 0;
+  const int g = int(plan.num_items < grid ? plan.num_items : grid);
+  const ScheduleKey key{head_dim, fused ? 1 : 0, int(plan.n_qtiles), len, hq, plan.pair_heads ? 1 : 0,
+                        fused ? S : 0, fused ? W : 0, fused ? n_obs : 0, g, int(plan.num_items)};
+  const lt::AttnSchedule& sched = attn_schedule(key, kStaticSchedule && plan.qt_band == 0);
+  if (!sched.used) return LT_OK;
+  *used = 1;
+  if (!off || !item || capacity < plan.num_items) return LT_ERR_INVALID_ARG;
+  for (int c = 0; c <= g; ++c) off[c] = sched.off[c];
+  for (long long t = 0; t < plan.num_items; ++t) item[t] = sched.item[t];
+  return LT_OK;
 }
 
 lt_status lt_prefill_attn(const lt_shape* shape, const void* Q, const void* K, const void* V, void* O, float* LSE,
