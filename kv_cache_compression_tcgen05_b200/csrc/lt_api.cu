@@ -228,6 +228,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // Long prefills: the attention's work items in q-tile bands, KV head by KV head.
 constexpr bool kBandedOrder = true;
+// Packed batches: the attention's work items sequence by sequence, KV head by KV head.
+constexpr bool kSeqMajorOrder = true;
 // Short single-sequence prefills: the static longest-first item schedule below.
 constexpr bool kStaticSchedule = true;
 
@@ -450,6 +452,7 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
   p.n_qtiles = int(n_qtiles);
   p.pair_heads = pair_heads ? 1 : 0;
   p.qt_band = int(qt_band);
+  p.seq_major = (kSeqMajorOrder && pair_heads && qt_band == 0 && shape->batch > 1) ? 1 : 0;
   p.num_items = int(num_items);
   p.cu_seqlens = shape->cu_seqlens;
   p.O = static_cast<__nv_bfloat16*>(O);
