@@ -276,6 +276,8 @@ FUSED = [
     # schedule, over q-tile pairs of one head (odd group) and over head pairs.
     dict(seqlens=(8000,), hq=12, hkv=4, d=64, S=4, W=700, n_obs=100),
     dict(seqlens=(5000,), hq=16, hkv=4, d=128, S=4, W=1500, n_obs=128),
+    # One long sequence with an odd group: banded q-tile pairs, ragged last pair.
+    dict(seqlens=(15000,), hq=10, hkv=2, d=64, S=4, W=3000, n_obs=100),
 ]
 
 

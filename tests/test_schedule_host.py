@@ -112,9 +112,12 @@ def test_long_and_tiny_launches_keep_their_orders():
     # Fewer items than CTAs: one item per CTA already.
     n, sched = lt.lt_attn_schedule(64, 256, 2, 1, 148)
     assert sched is None and n == 2
-    # More items than the schedule holds (1536): the snake order.
+    # More items than the schedule holds (1536): the snake order (an odd group over
+    # 32 768 tokens, and an even group too short for bands).
     n, sched = lt.lt_attn_schedule(128, 32768, 40, 8, 148, S=4, W=2044, n_obs=128, fused=True)
     assert sched is None and n == 128 * 40
+    n, sched = lt.lt_attn_schedule(64, 16384, 32, 16, 148, S=4, W=1020, n_obs=64, fused=True)
+    assert sched is None and n == 128 * 16
 
 
 def test_schedule_argument_errors():
