@@ -109,6 +109,10 @@ __device__ __forceinline__ void softmax_merge(float& m1, float& l1, float (&o1)[
 
 template <int D>
 __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeParams p) {
+  // Programmatic dependent launch: this kernel may start while the previous
+  // one in the stream finishes; it waits for it before touching memory.
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int E = 8;           // elements of a row per lane (one 16-byte load)
   constexpr int LPR = D / E;     // lanes per row
   constexpr int GPW = 32 / LPR;  // row groups per warp
@@ -308,6 +312,8 @@ __host__ __device__ inline size_t decode_splitk_floats(int batch, int hq, int he
 
 template <int D>
 __global__ void __launch_bounds__(kDecodeThreads) decode_splitk_kernel(const DecodeParams p, float* part) {
+  pdl_wait();
+  pdl_launch_dependents();
   constexpr int E = 8;           // elements of a row per lane (one 16-byte load)
   constexpr int LPR = D / E;     // lanes per row
   constexpr int GPW = 32 / LPR;  // row groups per warp
@@ -479,6 +485,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_splitk_kernel(const Dec
 template <int D>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const float* part, int hq, int splits, __nv_bfloat16* O,
                                                          float* LSE) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int h = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
   const float* src = part + (size_t(b) * hq + h) * splits * (D + 2);
   float M = -INFINITY;

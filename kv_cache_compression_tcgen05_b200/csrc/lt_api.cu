@@ -884,13 +884,15 @@ lt_status launch_decode(lt::DecodeParams& p, int head_dim, int max_len, float so
   cfg.blockDim = dim3(lt::kDecodeThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = p.splits;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlaps the previous kernel's tail
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = head_dim == 64 ? cudaLaunchKernelEx(&cfg, lt::decode_kernel<64>, p)
                                        : cudaLaunchKernelEx(&cfg, lt::decode_kernel<128>, p);
   return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
@@ -997,14 +999,18 @@ lt_status launch_decode_splitk(const void* q, const void* K, const void* V, cons
   p.scale_log2 = resolve_scale(softmax_scale, head_dim) * kLog2e;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const dim3 grid(hkv * splits, batch, 1), mgrid(hq, batch, 1);
+  // Both launches programmatic: each may start while the kernel before it
+  // finishes, and waits for it before touching memory.
+  cudaError_t e;
   if (head_dim == 64) {
-    lt::decode_splitk_kernel<64><<<grid, lt::kDecodeThreads, 0, s>>>(p, part);
-    lt::decode_merge_kernel<64><<<mgrid, 64, 0, s>>>(part, hq, splits, p.O, LSE);
+    e = launch_pdl(lt::decode_splitk_kernel<64>, grid, dim3(lt::kDecodeThreads), 0, s, p, part);
+    if (e == cudaSuccess) e = launch_pdl(lt::decode_merge_kernel<64>, mgrid, dim3(64), 0, s, part, hq, splits, p.O, LSE);
   } else {
-    lt::decode_splitk_kernel<128><<<grid, lt::kDecodeThreads, 0, s>>>(p, part);
-    lt::decode_merge_kernel<128><<<mgrid, 128, 0, s>>>(part, hq, splits, p.O, LSE);
+    e = launch_pdl(lt::decode_splitk_kernel<128>, grid, dim3(lt::kDecodeThreads), 0, s, p, part);
+    if (e == cudaSuccess)
+      e = launch_pdl(lt::decode_merge_kernel<128>, mgrid, dim3(128), 0, s, part, hq, splits, p.O, LSE);
   }
-  return cudaGetLastError() == cudaSuccess ? LT_OK : LT_ERR_CUDA;
+  return (e == cudaSuccess && cudaGetLastError() == cudaSuccess) ? LT_OK : LT_ERR_CUDA;
 }
 
 }  // namespace
