@@ -350,3 +350,39 @@ def test_fused_ratio_accumulate_mode(d):
     assert (rc - (r1 + 0.25)).abs().max().item() <= 1e-6
     with pytest.raises(ValueError):
         lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, accumulate=True, **kw)
+
+
+def _schedule_sweep_specs():
+    """Seeded single-sequence shapes whose launches take the static longest-first
+    schedule (more work items than SMs, at most 1536): one per group size 1..6,
+    both head dims, ragged lengths."""
+    rng = np.random.default_rng(2024)
+    specs = []
+    for hq, hkv in [(16, 16), (32, 16), (24, 8), (32, 8), (40, 8), (12, 2)]:
+        for _ in range(200):
+            d = int(rng.choice([64, 128]))
+            n = int(rng.integers(1200, 4200))
+            S, W, n_obs = int(rng.integers(0, 9)), int(rng.integers(64, 1500)), int(rng.integers(16, 129))
+            _, sched = lt.lt_attn_schedule(d, n, hq, hkv, 148, S=S, W=W, n_obs=n_obs, fused=True)
+            if sched is not None:
+                specs.append(dict(seqlens=(n,), hq=hq, hkv=hkv, d=d, S=S, W=W, n_obs=n_obs))
+                break
+    return specs
+
+
+@pytest.mark.parametrize("spec", _schedule_sweep_specs(), ids=lambda s: f"{s['seqlens'][0]}-{s['hq']}x{s['hkv']}-d{s['d']}")
+def test_static_schedule_parity_sweep(spec):
+    """Launches that run the static schedule: plain and fused attention against the
+    oracle on every row, the fused ratio against the oracle, and the fused kernel's
+    O and LSE equal to the plain kernel's bit for bit."""
+    cfg = synth.custom(seqlens=spec["seqlens"], hq=spec["hq"], hkv=spec["hkv"], d=spec["d"], S=spec["S"],
+                       W=spec["W"], n_obs=spec["n_obs"], seed=77)
+    from tests.gpu_common import gpu_fused
+    Q, K, V = synth.layer_inputs(cfg, 0, "cuda")
+    O1, L1 = gpu_attention(cfg, Q, K, V)
+    O2, L2, r = gpu_fused(cfg, Q, K, V)
+    torch.cuda.synchronize()
+    assert torch.equal(O1, O2) and torch.equal(L1, L2)
+    rel, lse_err = check_attention(cfg, Q, K, V, O2, L2)
+    assert rel <= O_REL_L2 and lse_err <= LSE_ABS, (rel, lse_err)
+    assert np.abs(r.cpu().numpy() - oracle_ratio(cfg, Q, K)).max() <= RATIO_ABS
