@@ -62,8 +62,7 @@ struct AttnParams {
   int group;        // hq / hkv
   int n_qtiles;     // ceil(max_seqlen / 128)
   int pair_heads;   // 1: an item pairs two heads; 0: it pairs two q-tiles
-  int qt_band;      // > 0 (with pair_heads): items ordered by q-tile bands of this many tiles, KV head by KV head
-  int seq_major;    // 1 (with pair_heads, qt_band 0): sequence by sequence, KV head by KV head
+  int qt_band;      // > 0 (with pair_heads): items ordered by sequence, then q-tile bands of this many tiles, KV head by KV head
   int num_items;
   const int32_t* cu_seqlens;  // device [batch+1] or null (one sequence)
   __nv_bfloat16* O;
@@ -159,47 +158,25 @@ __device__ __forceinline__ void seq_bounds(const AttnParams& p, int b, int& star
 // Items are ordered heaviest first; the items of one q position are consecutive
 // (heads of a sequence next to each other, so concurrent CTAs share K/V in L2).
 __device__ __forceinline__ bool attn_decode(const AttnParams& p, int t, AttnItem& it) {
-  if (p.pair_heads && p.seq_major) {
-    // Packed batches: sequence by sequence, within a sequence KV head by KV
-    // head, heaviest q-tile first: the CTAs running at the same time stream
-    // one KV head of one sequence (which then stays in L2) instead of every
-    // sequence's K/V at once.
+  if (p.pair_heads && p.qt_band > 0) {
+    // Banded order: sequence by sequence (a packed batch), q-tiles in bands of
+    // qt_band (heaviest band first), and within a band one KV head after
+    // another, so the CTAs running at the same time stream the same KV head's
+    // K/V (which then stays in L2) instead of every KV head's (and every
+    // sequence's) at once.  A long single sequence takes bands of about one
+    // wave of the grid, a packed batch one band per sequence.
     const int ppk = p.group >> 1;                       // head pairs per KV head
-    const int per_kh = p.n_qtiles * ppk;
-    const int per_seq = per_kh * p.hkv;
+    const int per_kh = p.qt_band * ppk;
+    const int per_band = per_kh * p.hkv;
+    const int per_seq = ((p.n_qtiles + p.qt_band - 1) / p.qt_band) * per_band;
     it.b = t / per_seq;
     int rem = t - it.b * per_seq;
+    const int band = rem / per_band;
+    rem -= band * per_band;
     const int kh = rem / per_kh;
     rem -= kh * per_kh;
     const int qin = rem / ppk;
     const int hp = kh * ppk + (rem - qin * ppk);
-    const int qt = p.n_qtiles - 1 - qin;
-    seq_bounds(p, it.b, it.start, it.len);
-    it.h[0] = 2 * hp;
-    it.h[1] = 2 * hp + 1;
-    it.qt[0] = it.qt[1] = qt;
-    it.n[0] = it.n[1] = qt + 1;
-    it.hasB = true;
-    it.kh = kh;
-    return qt * 128 < it.len;
-  }
-  if (p.pair_heads && p.qt_band > 0) {
-    // Long sequences: q-tiles in bands of qt_band (heaviest band first), and
-    // within a band one KV head after another, so the CTAs running at the same
-    // time stream the same KV head's K/V (which then stays in L2) instead of
-    // every KV head's at once.
-    const int ppk = p.group >> 1;                       // head pairs per KV head
-    const int per_qt = p.batch * ppk;
-    const int per_kh = p.qt_band * per_qt;
-    const int per_band = per_kh * p.hkv;
-    const int band = t / per_band;
-    int rem = t - band * per_band;
-    const int kh = rem / per_kh;
-    rem -= kh * per_kh;
-    const int qin = rem / per_qt;
-    rem -= qin * per_qt;
-    it.b = rem / ppk;
-    const int hp = kh * ppk + (rem - it.b * ppk);
     const int qt = p.n_qtiles - 1 - (band * p.qt_band + qin);
     if (qt < 0) return false;                           // the last band's unused places
     seq_bounds(p, it.b, it.start, it.len);

@@ -340,13 +340,14 @@ void build_schedule(const ScheduleKey& k, lt::AttnSchedule& out) {
 // The schedule for a launch: the snake order (used = 0) unless the launch is
 // one sequence of known length with at most kSchedMaxItems items; the last
 // shape's schedule is kept per host thread.
-// The attention launch's work items: q-tile bands for a long single sequence
-// (see attn_decode) and the item count.  Band order for a single sequence with
-// at least two bands of q-tiles, a band being about one wave of the grid on one
-// KV head.  Shorter prefills keep the plain heaviest-first order, which
-// balances their tail, and so do packed batches: sequences of different
-// lengths leave the bands' waves partly empty (measured 5.6% slower on the
-// batched workload, against 6.9% faster on a single 131 072-token sequence).
+// The attention launch's work items: q-tile bands (see attn_decode) and the
+// item count.  A single sequence with at least two bands of q-tiles takes bands
+// of about one wave of the grid on one KV head (6.9% faster on a 131 072-token
+// sequence); shorter single sequences keep the plain heaviest-first order,
+// which balances their tail.  A packed batch (even group) takes one band per
+// sequence: sequence by sequence, KV head by KV head (9.5% faster on the
+// batched workload; bands of one wave with the sequences interleaved measured
+// 5.6% slower, their waves partly empty with sequences of different lengths).
 struct AttnPlan {
   bool pair_heads;
   long long n_qtiles, qt_band, num_items;
@@ -360,6 +361,10 @@ AttnPlan attn_plan(int batch, int hq, int hkv, int max_len, int sm_count) {
   if (pl.pair_heads && kBandedOrder && batch == 1) {
     const long long band = std::max<long long>(1, sm_count / ((long long)batch * (group / 2)));
     if (pl.n_qtiles >= 2 * band) pl.qt_band = band;
+  } else if (pl.pair_heads && kSeqMajorOrder && batch > 1) {
+    // Packed batch: one band of all q-tiles per sequence, i.e. sequence by
+    // sequence and within one KV head by KV head.
+    pl.qt_band = pl.n_qtiles;
   }
   if (pl.qt_band > 0)
     pl.num_items = ((pl.n_qtiles + pl.qt_band - 1) / pl.qt_band) * pl.qt_band * hkv * batch * (group / 2);
@@ -452,7 +457,6 @@ static lt_status launch_attention(const lt_shape* shape, const void* Q, const vo
   p.n_qtiles = int(n_qtiles);
   p.pair_heads = pair_heads ? 1 : 0;
   p.qt_band = int(qt_band);
-  p.seq_major = (kSeqMajorOrder && pair_heads && qt_band == 0 && shape->batch > 1) ? 1 : 0;
   p.num_items = int(num_items);
   p.cu_seqlens = shape->cu_seqlens;
   p.O = static_cast<__nv_bfloat16*>(O);
