@@ -421,37 +421,48 @@ def run_ours(args, cfg, rank, world):
         ranks_agree = all(torch.equal(o, orders[0]) for o in orders)
 
     # Beside the step: the plain attention and the separate ratio pass per
-    # layer (all layers twice for short steps, the first four once for long ones).
+    # layer (all layers for short steps, the first four for long ones), captured
+    # in one CUDA graph with external timing events around every launch, so the
+    # times are the device's alone (no host gaps between eager launches).  The
+    # fused kernel is timed in the same graph (its accumulate form, as in the
+    # step), right after the plain one on the same inputs, so the ratio's
+    # overhead compares the two kernels under the same conditions (clock,
+    # power, L2).  Medians over the layers (every layer twice for short steps).
     kw = pf.kw
     side_layers = list(range(min(cfg.layers, 4))) if long_step else list(range(cfg.layers))
-    # The fused kernel is timed in the same loop (its zeroing form), right after
-    # the plain one on the same inputs, so the ratio's overhead compares the
-    # two kernels under the same conditions (clock, power, L2).
     attn_ev, ratio_ev, fused_eager_ev = [], [], []
     ratio_out = torch.empty_like(pf.ratio[0])
-    for rep in range(2 if not long_step else 1):
-        for l in side_layers:
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True, external=True)
+
+    g_side = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_side, stream=stream):
+        for l in side_layers * (1 if long_step else 2):
             Q, K, V = pf.layers[l]
-            e0, e1, e2, e3 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
-            e0.record()
-            lt.lt_prefill_attn(Q, K, V, out=pf.O, lse=pf.LSE, **kw)
-            e1.record()
-            lt.lt_lazy_ratio(Q, K, pf.LSE, cfg.S, cfg.W, cfg.n_obs, out=ratio_out, **kw)
-            e2.record()
+            e0, e1, e2, e2b, e3 = ev(), ev(), ev(), ev(), ev()
+            e0.record(stream)
+            lt.lt_prefill_attn(Q, K, V, out=pf.O, lse=pf.LSE, stream=stream, **kw)
+            e1.record(stream)
+            lt.lt_lazy_ratio(Q, K, pf.LSE, cfg.S, cfg.W, cfg.n_obs, out=ratio_out, stream=stream, **kw)
+            e2.record(stream)
             ratio_out.zero_()      # outside the fused launch's events (accumulate form, as in the step)
-            e2b = torch.cuda.Event(enable_timing=True)
-            e2b.record()
+            e2b.record(stream)
             lt.lt_prefill_attn_ratio(Q, K, V, cfg.S, cfg.W, cfg.n_obs, out=pf.O, lse=pf.LSE, ratio=ratio_out,
-                                     accumulate=True, **kw)
-            e3.record()
-            if rep > 0 or long_step and l > 0:
+                                     accumulate=True, stream=stream, **kw)
+            e3.record(stream)
+            if not long_step or l > 0:
                 attn_ev.append((e0, e1))
                 ratio_ev.append((e1, e2))
                 fused_eager_ev.append((e2b, e3))
+    with torch.cuda.stream(stream):
+        for _ in range(1 if long_step else 2):     # the last replay's events are read
+            g_side.replay()
     torch.cuda.synchronize()
-    t_attn = statistics.mean(a.elapsed_time(b) for a, b in attn_ev) * 1e-3
-    t_ratio = statistics.mean(a.elapsed_time(b) for a, b in ratio_ev) * 1e-3
-    t_fused_eager = statistics.mean(a.elapsed_time(b) for a, b in fused_eager_ev) * 1e-3
+    t_attn = statistics.median(a.elapsed_time(b) for a, b in attn_ev) * 1e-3
+    t_ratio = statistics.median(a.elapsed_time(b) for a, b in ratio_ev) * 1e-3
+    t_fused_eager = statistics.median(a.elapsed_time(b) for a, b in fused_eager_ev) * 1e-3
+    del g_side
     kv = pf.kv_report(step_alloc)
 
     if args.kernels_only:
