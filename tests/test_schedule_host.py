@@ -108,7 +108,7 @@ def test_gqa1p2b_fused_schedule_is_used_and_beats_snake():
 def test_long_and_tiny_launches_keep_their_orders():
     # 131 072 tokens: banded item order (no static schedule).
     n, sched = lt.lt_attn_schedule(128, 131072, 32, 8, 148, S=4, W=4092, n_obs=128, fused=True)
-    assert sched is None and n == 16576     # 1024 q-tiles in bands of 37, 8 KV heads, 2 head pairs each
+    assert sched is None and n == 16576     # 1024 q-tiles in 14 bands of 74, 8 KV heads, 2 head pairs each
     # Fewer items than CTAs: one item per CTA already.
     n, sched = lt.lt_attn_schedule(64, 256, 2, 1, 148)
     assert sched is None and n == 2
