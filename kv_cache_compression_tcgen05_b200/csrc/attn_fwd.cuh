@@ -7,29 +7,36 @@
 // built for B200 (the library runs it at head_dim 128; head_dim 64 runs the
 // variant in attn_fwd64.cuh, whose P has TMEM columns of its own):
 //
-//   * persistent: one CTA per SM walks a list of work items, heaviest first,
-//     snake-ordered across CTAs.  A work item is two 128-row query tiles that
-//     read the same K/V stream: two query heads of one KV head at the same
-//     q-tile when the GQA group is even, otherwise two consecutive q-tiles of
-//     one head (the earlier tile then skips the last key tile).
-//   * warp-specialised, 10 working warps (12 launched):
-//       warp 0      TMA producer: the item's two Q tiles (double buffered) and
+//   * persistent: one CTA per SM walks a list of work items.  A work item is
+//     two 128-row query tiles that read the same K/V stream: two query heads
+//     of one KV head at the same q-tile when the GQA group is even, otherwise
+//     two consecutive q-tiles of one head (the earlier tile then skips the last
+//     key tile).  The order (attn_decode): heaviest q-tile first; for a long
+//     single sequence and for packed batches, sequence by sequence and in
+//     q-tile bands KV head by KV head (concurrent CTAs share one KV head's K/V
+//     in L2); CTAs take items in a snake order, or, for a short single
+//     sequence, as a longest-first assignment computed on the host (the
+//     AttnSchedule parameter).
+//   * warp-specialised, three warpgroups (12 warps, 10 working); setmaxnreg
+//     gives the softmax warpgroups 184 registers a thread and the third 136:
+//       warps 0..3  softmax of tile A, warps 4..7 softmax of tile B: thread =
+//                   query row = TMEM lane.  tcgen05.ld of the 128 scores, causal
+//                   mask on the diagonal tile, running max in the log2 domain
+//                   (the O accumulator is rescaled only when the max grows by
+//                   more than 2^8; exact, because O and l share the stale max),
+//                   exp2 with the scale/shift and row sum in packed two-lane
+//                   fp32, bf16 P written back over the scores in TMEM with
+//                   tcgen05.st (P is the A operand of O += P V, read from TMEM);
+//                   epilogue O / l and LSE = (m + log2 l) ln 2, written once;
+//       warp 8      TMA producer: the item's two Q tiles (double buffered) and
 //                   a ring of K/V tiles (128 keys x d, 128-byte swizzle);
-//       warp 1      owns the TMEM allocation; one thread issues every
+//       warp 9      owns the TMEM allocation; one thread issues every
 //                   tcgen05.mma in the order
 //                       S_A(0), S_B(0), [PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)]
 //                   so the tensor core works on one tile while the other
 //                   tile's softmax runs (shared-memory descriptors are built
 //                   once and advanced by address/16, so the single issuing
-//                   thread spends little per instruction);
-//       warps 2..5  softmax of tile A, warps 6..9 softmax of tile B: thread =
-//                   query row = TMEM lane.  tcgen05.ld of the 128 scores, causal
-//                   mask on the diagonal tile, running max in the log2 domain
-//                   (the O accumulator is rescaled only when the max grows by
-//                   more than 2^8; exact, because O and l share the stale max),
-//                   exp2, bf16 P written back over the scores in TMEM with
-//                   tcgen05.st (P is the A operand of O += P V, read from TMEM);
-//                   epilogue O / l and LSE = (m + log2 l) ln 2, written once.
+//                   thread spends little per instruction).
 //   * TMEM columns: [0,128) S/P of A, [128,256) S/P of B, [256,256+d) O of A,
 //     [256+d, 256+2d) O of B.  P overwrites the first half of its S columns.
 //     The MMAs of one thread execute in issue order, so S_X(j+1), issued after
