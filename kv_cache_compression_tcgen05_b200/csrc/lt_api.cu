@@ -230,6 +230,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr bool kBandedOrder = true;
 // Packed batches: the attention's work items sequence by sequence, KV head by KV head.
 constexpr bool kSeqMajorOrder = true;
+// Split-K decode: caches longer than this take the two-CTAs-a-SM kernel
+// (measured faster from 32 768 rows on, slower at 4096).
+constexpr int kDecodeSplitKDense = 8192;
 // Short single-sequence prefills: the static longest-first item schedule below.
 constexpr bool kStaticSchedule = true;
 
@@ -1006,11 +1009,15 @@ lt_status launch_decode_splitk(const void* q, const void* K, const void* V, cons
   // Both launches programmatic: each may start while the kernel before it
   // finishes, and waits for it before touching memory.
   cudaError_t e;
+  // Caches of more than kDecodeSplitKDense rows: two CTAs a SM.
+  const bool dense = max_len > kDecodeSplitKDense;
   if (head_dim == 64) {
-    e = launch_pdl(lt::decode_splitk_kernel<64>, grid, dim3(lt::kDecodeThreads), 0, s, p, part);
+    e = dense ? launch_pdl(lt::decode_splitk_kernel<64, 2>, grid, dim3(lt::kDecodeThreads), 0, s, p, part)
+              : launch_pdl(lt::decode_splitk_kernel<64, 1>, grid, dim3(lt::kDecodeThreads), 0, s, p, part);
     if (e == cudaSuccess) e = launch_pdl(lt::decode_merge_kernel<64>, mgrid, dim3(64), 0, s, part, hq, splits, p.O, LSE);
   } else {
-    e = launch_pdl(lt::decode_splitk_kernel<128>, grid, dim3(lt::kDecodeThreads), 0, s, p, part);
+    e = dense ? launch_pdl(lt::decode_splitk_kernel<128, 2>, grid, dim3(lt::kDecodeThreads), 0, s, p, part)
+              : launch_pdl(lt::decode_splitk_kernel<128, 1>, grid, dim3(lt::kDecodeThreads), 0, s, p, part);
     if (e == cudaSuccess)
       e = launch_pdl(lt::decode_merge_kernel<128>, mgrid, dim3(128), 0, s, part, hq, splits, p.O, LSE);
   }
