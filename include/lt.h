@@ -410,12 +410,12 @@ lt_status lt_decode_attn(const void* q, const void* K, const void* V, const int3
                          float* LSE, float softmax_scale, lt_stream stream);
 
 /*
- * lt_decode_attn for long caches: the same decode step (same arguments,
+ * lt_decode_attn split over many CTAs: the same decode step (same arguments,
  * layouts, results and errors, except head_dim 64/128 and the workspace),
- * with the rows of each (sequence, KV head) split over
- * ceil(max_len / 1024) CTAs (at most 128; any number, where lt_decode_attn's
- * cluster split stops at 16), so that a batch-1 decode over a few KV heads
- * keeps every SM streaming K/V.  Each CTA writes its partial softmax state
+ * with the rows of each (sequence, KV head) split over ceil(max_len / r) CTAs,
+ * r = ceil(max_len / 16) clamped to [256, 1024] rows (at most 128 CTAs; any
+ * number, where lt_decode_attn's cluster split stops at 16), so that a
+ * batch-1 decode over a few KV heads keeps every SM streaming K/V.  Each CTA writes its partial softmax state
  * (running max and sum, unnormalised output of every query head) to
  * `workspace`; a second kernel merges the splits of each head in split order
  * (deterministic).  workspace: caller-allocated device memory of at least

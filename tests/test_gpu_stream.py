@@ -282,6 +282,6 @@ def test_splitk_decode_rejects_a_small_workspace():
     K = torch.zeros((1, 5000, 2, 64), dtype=torch.bfloat16, device="cuda")
     ln = torch.full((1,), 5000, dtype=torch.int32, device="cuda")
     need = lt.lt_decode_splitk_workspace_bytes(1, 4, 64, 5000)
-    assert need == 4 * 5 * (64 + 2) * 4          # 4 heads, ceil(5000 / 1024) = 5 splits
+    assert need == 4 * 16 * (64 + 2) * 4         # 4 heads; splits of ceil(5000 / 16) = 313 rows: 16 splits
     with pytest.raises(lt.LtError):
         lt.lt_decode_attn_splitk(q, K, K, ln, workspace=torch.empty(need - 16, dtype=torch.uint8, device="cuda"))
