@@ -432,9 +432,12 @@ def run_ours(args, cfg, rank, world):
     side_layers = list(range(min(cfg.layers, 4))) if long_step else list(range(cfg.layers))
     attn_ev, ratio_ev, fused_eager_ev = [], [], []
     ratio_out = torch.empty_like(pf.ratio[0])
+    side_events = []   # every event the graph records into lives until the graph is released
 
     def ev():
-        return torch.cuda.Event(enable_timing=True, external=True)
+        e = torch.cuda.Event(enable_timing=True, external=True)
+        side_events.append(e)
+        return e
 
     g_side = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_side, stream=stream):
@@ -463,6 +466,7 @@ def run_ours(args, cfg, rank, world):
     t_ratio = statistics.median(a.elapsed_time(b) for a, b in ratio_ev) * 1e-3
     t_fused_eager = statistics.median(a.elapsed_time(b) for a, b in fused_eager_ev) * 1e-3
     del g_side
+    del side_events
     kv = pf.kv_report(step_alloc)
 
     if args.kernels_only:
