@@ -213,3 +213,13 @@ def test_queue_and_pool_calls_reject_bad_arguments():
     # nothing to compact: succeeds without a device
     assert lib.lt_compact_kv_layers(ctypes.byref(s), FAKE, FAKE, 4, None, 0, 4, 8, None, None, None, None) == lt.LT_OK
     assert lib.lt_selftest_wait_timeout(0, None) == INV
+
+
+@pytest.mark.parametrize("max_len,splits", [(1, 1), (256, 1), (1024, 4), (4096, 16), (5000, 16), (8192, 16),
+                                            (16384, 16), (32768, 32), (131072, 128), (1 << 20, 128)])
+def test_splitk_workspace_follows_the_split_rule(max_len, splits):
+    """The split-K decode splits each (sequence, KV head) into ceil(max_len / r)
+    CTAs, r = ceil(max_len / 16) clamped to [256, 1024], at most 128; its
+    workspace holds batch x hq x splits x (head_dim + 2) floats (host call)."""
+    for batch, hq, d in [(1, 32, 128), (3, 8, 64)]:
+        assert lt.lt_decode_splitk_workspace_bytes(batch, hq, d, max_len) == batch * hq * splits * (d + 2) * 4
