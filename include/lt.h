@@ -37,7 +37,11 @@
  *     16-byte aligned.  When total_tokens is 0 the token-indexed inputs and
  *     outputs (Q, K, V, O, LSE) are not accessed and may be null.
  *   - Calls that take a stream only enqueue work on it (they never synchronise
- *     the device); their outputs are ready when the stream reaches them.  They
+ *     the device); their outputs are ready when the stream reaches them.  Most
+ *     kernels are launched with programmatic dependent launch: one may start
+ *     while the kernel before it in the stream is finishing, and waits for that
+ *     kernel's completion (all its writes visible) before it touches memory, so
+ *     to the caller this is ordinary stream order.  They
  *     launch on the calling thread's current CUDA device: the stream and every
  *     device pointer must belong to that device (the library cannot check a
  *     pointer's device; the Python binding checks its tensors').
