@@ -12,13 +12,13 @@ heaviest first), costing its key tiles (the two tiles run side by side) plus one
 tile of fixed work, and with the fused ratio two more tiles per key tile that
 holds a sink or an observed row's first window key.
 """
+import ctypes
+
 import numpy as np
 import pytest
 
 import kv_cache_compression_tcgen05_b200 as lt
-from kv_cache_compression_tcgen05_b200.binding import library, LT_ERR_INVALID_ARG
-
-import ctypes
+from kv_cache_compression_tcgen05_b200.binding import LT_ERR_INVALID_ARG, library
 
 
 def masked_tiles(qt, n, S, W, n_obs):
